@@ -1,0 +1,389 @@
+// C ABI of libmoba.so: argument validation, the host-side plan (block counts, query chunks,
+// workspace layout), launch sequencing and optional per-kernel event timing. Every step of the
+// computation runs in the kernels; this file only sizes and orders them.
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/moba.h"
+#include "common.cuh"
+#include "launch.h"
+
+using namespace moba;
+
+namespace {
+
+constexpr size_t kPartialBudgetBytes = 16ull << 30;  // per-chunk partial outputs + routing lists
+constexpr int kNumClasses = 8;
+enum KernelClass { kCentroid = 0, kGate, kRouteCount, kRouteScan, kRouteScatter, kAttn, kMerge, kPlan };
+
+std::atomic<long long> g_launches{0};
+
+// ------------------------------------------------------------------------------- timing hooks
+struct Timing {
+  std::mutex mu;
+  bool enabled = false;
+  double ms[kNumClasses] = {0};
+  long long n[kNumClasses] = {0};
+  struct Pending { int cls; cudaEvent_t a, b; };
+  std::vector<Pending> pending;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) { cudaEvent_t e = pool.back(); pool.pop_back(); return e; }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+};
+Timing& timing() { static Timing t; return t; }
+
+struct Scope {  // brackets one kernel launch with events when timing is enabled
+  int cls; cudaStream_t s; cudaEvent_t a = nullptr, b = nullptr; bool on = false;
+  Scope(int c, cudaStream_t st) : cls(c), s(st) {
+    Timing& T = timing();
+    std::lock_guard<std::mutex> g(T.mu);
+    if (T.enabled) { on = true; a = T.get(); b = T.get(); cudaEventRecord(a, s); }
+  }
+  void done() {
+    g_launches.fetch_add(1);
+    if (!on) return;
+    cudaEventRecord(b, s);
+    Timing& T = timing();
+    std::lock_guard<std::mutex> g(T.mu);
+    T.pending.push_back({cls, a, b});
+  }
+};
+
+// ----------------------------------------------------------------------------------- device
+struct DevInfo { int ok = -1; int sms = 0; };
+int device_check(int* sms) {
+  static DevInfo info[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOBA_ERR_CUDA;
+  DevInfo& di = info[dev];
+  if (di.ok < 0) {
+    cudaDeviceProp p;
+    if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return MOBA_ERR_CUDA;
+    di.ok = (p.major == 10 && p.minor == 0) ? 1 : 0;
+    di.sms = p.multiProcessorCount;
+  }
+  if (sms) *sms = di.sms;
+  return di.ok ? MOBA_OK : MOBA_ERR_UNSUPPORTED;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------------------------- plan
+struct Chunk { int b0, nblk, T0, ntok; };
+struct Plan {
+  int T = 0, NB = 0, max_nb = 0;
+  std::vector<int> blk_len;  // per global block
+  std::vector<Chunk> chunks;
+  size_t max_rows = 0, max_entries = 0, max_tiles = 0;
+};
+
+int check_cu(int nseq, const int32_t* cu) {
+  if (nseq < 1 || nseq > 65535 || !cu) return MOBA_ERR_ARG;
+  if (cu[0] != 0) return MOBA_ERR_ARG;
+  for (int s = 0; s < nseq; ++s)
+    if (cu[s + 1] < cu[s]) return MOBA_ERR_ARG;
+  return MOBA_OK;
+}
+
+int check_shape(int Hq, int Hkv, int d, int B, int topk) {
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return MOBA_ERR_ARG;
+  if (B < 1 || topk < 1) return MOBA_ERR_ARG;
+  if (d != 64 && d != 128) return MOBA_ERR_UNSUPPORTED;
+  if (B % 64 != 0) return MOBA_ERR_UNSUPPORTED;
+  if (topk > kMaxTopk) return MOBA_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 256) return MOBA_ERR_UNSUPPORTED;
+  return MOBA_OK;
+}
+
+int make_plan(int nseq, const int32_t* cu, int Hq, int Hkv, int d, int B, int topk, Plan* P) {
+  P->T = cu[nseq];
+  P->blk_len.clear();
+  for (int s = 0; s < nseq; ++s) {
+    const int L = cu[s + 1] - cu[s];
+    const int nb = blocks_of(L, B);
+    if (nb > kMaxBlocksPerSeq) return MOBA_ERR_UNSUPPORTED;
+    P->max_nb = std::max(P->max_nb, nb);
+    for (int j = 0; j < nb; ++j) P->blk_len.push_back(std::min(B, L - j * B));
+  }
+  P->NB = static_cast<int>(P->blk_len.size());
+  if (static_cast<long long>(P->T) * Hq >= (1LL << 31) / 2) return MOBA_ERR_UNSUPPORTED;
+  if (P->max_nb > 65535) return MOBA_ERR_UNSUPPORTED;
+  // query chunks of whole blocks, so that partial rows (t, h, slot) fit the budget
+  const size_t row_bytes = static_cast<size_t>(d) * 2 + 4 + 4;
+  size_t max_rows = kPartialBudgetBytes / row_bytes;
+  const size_t per_tok = static_cast<size_t>(Hq) * topk;
+  max_rows = std::min<size_t>(max_rows, (1ull << 31) - 1);
+  P->chunks.clear();
+  int b = 0, t = 0;
+  while (b < P->NB) {
+    Chunk c{b, 0, t, 0};
+    while (b < P->NB) {
+      const size_t rows = static_cast<size_t>(c.ntok + P->blk_len[b]) * per_tok;
+      if (c.nblk > 0 && rows > max_rows) break;
+      if (rows >= (1ull << 31)) return MOBA_ERR_UNSUPPORTED;
+      c.ntok += P->blk_len[b];
+      c.nblk += 1;
+      ++b;
+    }
+    t += c.ntok;
+    P->chunks.push_back(c);
+    const size_t rows = static_cast<size_t>(c.ntok) * per_tok;
+    const size_t ent = static_cast<size_t>(c.ntok) * Hq * (topk - 1);
+    P->max_rows = std::max(P->max_rows, rows);
+    P->max_entries = std::max(P->max_entries, ent);
+    P->max_tiles = std::max(P->max_tiles, ent / kTile + static_cast<size_t>(Hkv) * P->NB + 1);
+  }
+  return MOBA_OK;
+}
+
+// --------------------------------------------------------------------------- workspace carve
+struct Layout {
+  size_t status, blk_off, blk_seq, blk_start, blk_len, cents, idx, counts, cursor, tiles,
+      entries, part_o, part_lse, total;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+Layout layout_of(const Plan& P, int nseq, int Hq, int Hkv, int d, int topk) {
+  Layout L;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t at = o; o = up256(o + bytes); return at; };
+  L.status = take(256);
+  L.blk_off = take(static_cast<size_t>(nseq + 1) * 4);
+  L.blk_seq = take(static_cast<size_t>(P.NB) * 4);
+  L.blk_start = take(static_cast<size_t>(P.NB) * 4);
+  L.blk_len = take(static_cast<size_t>(P.NB) * 4);
+  L.cents = take(static_cast<size_t>(P.NB) * Hkv * d * 4);
+  L.idx = take(static_cast<size_t>(Hq) * P.T * topk * 4);
+  L.counts = take(static_cast<size_t>(Hkv) * P.NB * 4);
+  L.cursor = take(static_cast<size_t>(Hkv) * P.NB * 4);
+  L.tiles = take(P.max_tiles * 16);
+  L.entries = take(std::max<size_t>(P.max_entries, 1) * 4);
+  L.part_o = take(P.max_rows * d * 2);
+  L.part_lse = take(P.max_rows * 4);
+  L.total = o;
+  return L;
+}
+
+template <class T>
+T* at(void* base, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(base) + off); }
+
+#define MOBA_LAUNCH(cls, stream, expr)                      \
+  do {                                                      \
+    Scope _sc((cls), (stream));                             \
+    cudaError_t _e = (expr);                                \
+    _sc.done();                                             \
+    if (_e != cudaSuccess) return MOBA_ERR_CUDA;            \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* moba_status_string(int status) {
+  switch (status) {
+    case MOBA_OK: return "MOBA_OK";
+    case MOBA_ERR_ARG: return "MOBA_ERR_ARG: invalid argument";
+    case MOBA_ERR_UNSUPPORTED: return "MOBA_ERR_UNSUPPORTED: shape or device not supported";
+    case MOBA_ERR_WORKSPACE: return "MOBA_ERR_WORKSPACE: workspace too small";
+    case MOBA_ERR_CUDA: return "MOBA_ERR_CUDA: CUDA call or kernel launch failed";
+    case MOBA_ERR_DEVICE_CHECK: return "MOBA_ERR_DEVICE_CHECK: device-side check failed";
+    case MOBA_ERR_TIMEOUT: return "MOBA_ERR_TIMEOUT: a bounded device wait ran out";
+    default: return "MOBA_UNKNOWN_STATUS";
+  }
+}
+
+int moba_version(void) { return (0 << 16) | (1 << 8) | 0; }
+
+size_t moba_workspace_bytes(int nseq, const int32_t* cu_seqlens_host, int Hq, int Hkv, int d,
+                            int block_size, int topk) {
+  if (check_cu(nseq, cu_seqlens_host) != MOBA_OK) return 0;
+  if (check_shape(Hq, Hkv, d, block_size, topk) != MOBA_OK) return 0;
+  Plan P;
+  if (make_plan(nseq, cu_seqlens_host, Hq, Hkv, d, block_size, topk, &P) != MOBA_OK) return 0;
+  return layout_of(P, nseq, Hq, Hkv, d, topk).total;
+}
+
+int moba_centroids(const void* k, const int32_t* cu_dev, const int32_t* cu_host, int nseq,
+                   int Hkv, int d, int block_size, float* centroids, void* stream) {
+  int st = check_cu(nseq, cu_host);
+  if (st != MOBA_OK) return st;
+  if (Hkv < 1 || block_size < 1) return MOBA_ERR_ARG;
+  if (d != 64 && d != 128) return MOBA_ERR_UNSUPPORTED;
+  if (block_size % 64 != 0) return MOBA_ERR_UNSUPPORTED;
+  Plan P;
+  if ((st = make_plan(nseq, cu_host, Hkv, Hkv, d, block_size, 1, &P)) != MOBA_OK) return st;
+  if (P.T == 0 || P.NB == 0) return MOBA_OK;
+  if (!k || !cu_dev || !centroids || !aligned16(k) || !aligned16(centroids)) return MOBA_ERR_ARG;
+  int sms = 0;
+  if ((st = device_check(&sms)) != MOBA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MOBA_LAUNCH(kCentroid, s,
+              launch_centroids(k, cu_dev, nseq, P.max_nb, Hkv, d, block_size, P.NB, sms, centroids, s));
+  return MOBA_OK;
+}
+
+int moba_gate_topk(const void* q, const float* centroids, const int32_t* cu_dev,
+                   const int32_t* cu_host, int nseq, int Hq, int Hkv, int d, int block_size,
+                   int topk, int32_t* block_idx, void* stream) {
+  int st = check_cu(nseq, cu_host);
+  if (st != MOBA_OK) return st;
+  if ((st = check_shape(Hq, Hkv, d, block_size, topk)) != MOBA_OK) return st;
+  Plan P;
+  if ((st = make_plan(nseq, cu_host, Hq, Hkv, d, block_size, topk, &P)) != MOBA_OK) return st;
+  if (P.T == 0) return MOBA_OK;
+  if (!q || !centroids || !cu_dev || !block_idx || !aligned16(q) || !aligned16(centroids) ||
+      !aligned16(block_idx))
+    return MOBA_ERR_ARG;
+  if ((st = device_check(nullptr)) != MOBA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MOBA_LAUNCH(kGate, s,
+              launch_gate(q, centroids, cu_dev, nseq, P.max_nb, P.T, Hq, Hkv, d, block_size, topk,
+                          block_idx, s));
+  return MOBA_OK;
+}
+
+int moba_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_dev,
+                  const int32_t* cu_host, int nseq, int Hq, int Hkv, int d, int block_size,
+                  int topk, float scale, const int32_t* block_idx_in, int32_t* block_idx_out,
+                  void* o, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_cu(nseq, cu_host);
+  if (st != MOBA_OK) return st;
+  if ((st = check_shape(Hq, Hkv, d, block_size, topk)) != MOBA_OK) return st;
+  if (!(scale > 0.f) || scale > 1e30f) return MOBA_ERR_ARG;
+  Plan P;
+  if ((st = make_plan(nseq, cu_host, Hq, Hkv, d, block_size, topk, &P)) != MOBA_OK) return st;
+  if (P.T == 0) return MOBA_OK;
+  if (!q || !k || !v || !cu_dev || !o || !lse || !workspace) return MOBA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return MOBA_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOBA_ERR_ARG;
+  if ((block_idx_in && !aligned16(block_idx_in)) || (block_idx_out && !aligned16(block_idx_out)))
+    return MOBA_ERR_ARG;
+  const Layout L = layout_of(P, nseq, Hq, Hkv, d, topk);
+  if (workspace_bytes < L.total) return MOBA_ERR_WORKSPACE;
+  int sms = 0;
+  if ((st = device_check(&sms)) != MOBA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  BlockTables tb;
+  tb.blk_off = at<int>(workspace, L.blk_off);
+  tb.blk_seq = at<int>(workspace, L.blk_seq);
+  tb.blk_start = at<int>(workspace, L.blk_start);
+  tb.blk_len = at<int>(workspace, L.blk_len);
+  int* status = at<int>(workspace, L.status);
+  int* n_tiles = status + 1;
+  int* counts = at<int>(workspace, L.counts);
+  int* cursor = at<int>(workspace, L.cursor);
+  int4* tiles = at<int4>(workspace, L.tiles);
+  int* entries = at<int>(workspace, L.entries);
+  void* part_o = at<void>(workspace, L.part_o);
+  float* part_lse = at<float>(workspace, L.part_lse);
+  float* cents = at<float>(workspace, L.cents);
+  const int NBK = Hkv * P.NB;
+
+  MOBA_LAUNCH(kPlan, s, launch_plan(cu_dev, nseq, block_size, P.NB, tb, counts, NBK, status, s));
+
+  const int32_t* idx = block_idx_in;
+  if (!idx) {
+    int32_t* idx_w = block_idx_out ? block_idx_out : at<int32_t>(workspace, L.idx);
+    MOBA_LAUNCH(kCentroid, s,
+                launch_centroids(k, cu_dev, nseq, P.max_nb, Hkv, d, block_size, P.NB, sms, cents, s));
+    MOBA_LAUNCH(kGate, s,
+                launch_gate(q, cents, cu_dev, nseq, P.max_nb, P.T, Hq, Hkv, d, block_size, topk,
+                            idx_w, s));
+    idx = idx_w;
+  } else if (block_idx_out && block_idx_out != block_idx_in) {
+    if (cudaMemcpyAsync(block_idx_out, block_idx_in, static_cast<size_t>(Hq) * P.T * topk * 4,
+                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return MOBA_ERR_CUDA;
+  }
+
+  for (const Chunk& c : P.chunks) {
+    MOBA_LAUNCH(kRouteCount, s,
+                launch_route_count(idx, tb, P.T, Hq, Hkv, topk, P.NB, c.b0, c.nblk, c.T0, P.max_nb,
+                                   counts, s));
+    MOBA_LAUNCH(kRouteScan, s, launch_route_scan(counts, NBK, cursor, tiles, n_tiles, s));
+    MOBA_LAUNCH(kRouteScatter, s,
+                launch_route_scatter(idx, tb, P.T, Hq, Hkv, topk, P.NB, c.b0, c.nblk, c.T0,
+                                     P.max_nb, cursor, entries, s));
+    AttnLaunch A;
+    A.q = q; A.k = k; A.v = v;
+    A.tiles = tiles; A.n_routed = n_tiles; A.entries = entries; A.tb = tb;
+    A.part_o = part_o; A.part_lse = part_lse; A.status = status;
+    A.T = P.T; A.H = Hq; A.G = Hkv; A.d = d; A.B = block_size; A.topk = topk; A.NB = P.NB;
+    A.b0 = c.b0; A.nblk = c.nblk; A.T0 = c.T0; A.scale = scale;
+    const long long P128 = (block_size + kTile - 1) / kTile;
+    const long long items = static_cast<long long>(P.max_tiles) + P128 * c.nblk * Hq;
+    A.grid = static_cast<int>(std::min<long long>(sms, items));
+    MOBA_LAUNCH(kAttn, s, launch_attention(A, s));
+    MOBA_LAUNCH(kMerge, s,
+                launch_merge(part_o, part_lse, cu_dev, nseq, P.T, Hq, d, block_size, topk, c.T0,
+                             c.ntok, o, lse, s));
+  }
+  return MOBA_OK;
+}
+
+int moba_device_status(const void* workspace, void* stream) {
+  if (!workspace) return MOBA_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOBA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOBA_ERR_CUDA;
+  if (word == 0) return MOBA_OK;
+  if (word == kDevTimeoutAttn) return MOBA_ERR_TIMEOUT;
+  return MOBA_ERR_DEVICE_CHECK;
+}
+
+int moba_timing_enable(int enable) {
+  Timing& T = timing();
+  std::lock_guard<std::mutex> g(T.mu);
+  T.enabled = enable != 0;
+  return MOBA_OK;
+}
+
+int moba_timing_reset(void) {
+  Timing& T = timing();
+  std::lock_guard<std::mutex> g(T.mu);
+  for (auto& p : T.pending) {
+    cudaEventSynchronize(p.b);
+    T.pool.push_back(p.a);
+    T.pool.push_back(p.b);
+  }
+  T.pending.clear();
+  for (int c = 0; c < kNumClasses; ++c) { T.ms[c] = 0; T.n[c] = 0; }
+  return MOBA_OK;
+}
+
+int moba_timing_read(double* ms_per_class, long long* launches_per_class, int n) {
+  Timing& T = timing();
+  std::lock_guard<std::mutex> g(T.mu);
+  for (auto& p : T.pending) {
+    if (cudaEventSynchronize(p.b) != cudaSuccess) return MOBA_ERR_CUDA;
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, p.a, p.b);
+    T.ms[p.cls] += ms;
+    T.n[p.cls] += 1;
+    T.pool.push_back(p.a);
+    T.pool.push_back(p.b);
+  }
+  T.pending.clear();
+  for (int c = 0; c < kNumClasses && c < n; ++c) {
+    if (ms_per_class) ms_per_class[c] = T.ms[c];
+    if (launches_per_class) launches_per_class[c] = T.n[c];
+  }
+  return kNumClasses;
+}
+
+long long moba_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

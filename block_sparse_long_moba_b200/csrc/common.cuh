@@ -1,0 +1,45 @@
+// Shared definitions of the MoBA kernels (device side) and their host launchers.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace moba {
+
+constexpr int kTile = 128;           // query rows per attention tile, keys per key sub-tile
+constexpr int kMaxTopk = 64;
+constexpr int kMaxBlocksPerSeq = 32768;
+constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s per bounded device wait
+
+// Device status word codes (written with atomicCAS(word, 0, code); first failure wins).
+constexpr int kDevTimeoutAttn = 0x101;
+
+// Block tables built on the device from cu_seqlens (workspace resident).
+struct BlockTables {
+  int* blk_off;    // [nseq + 1] first global block of each sequence
+  int* blk_seq;    // [NB] sequence of each global block
+  int* blk_start;  // [NB] first token of each block (absolute)
+  int* blk_len;    // [NB] number of keys in each block
+};
+
+// Number of key blocks of a sequence of length L.
+__host__ __device__ __forceinline__ int blocks_of(int L, int B) { return (L + B - 1) / B; }
+
+// Cooperative (whole CTA) computation of the first global block of sequence s:
+// sum over s' < s of ceil(len_s' / B). Every thread of the CTA must call it.
+__device__ __forceinline__ int seq_block_base(const int32_t* cu, int s, int B, int* red_smem) {
+  int acc = 0;
+  for (int x = threadIdx.x; x < s; x += blockDim.x) acc += blocks_of(cu[x + 1] - cu[x], B);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  const int warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red_smem[warp] = acc;
+  __syncthreads();
+  int tot = 0;
+  for (int w = 0; w < nw; ++w) tot += red_smem[w];
+  __syncthreads();
+  return tot;
+}
+
+}  // namespace moba

@@ -1,0 +1,55 @@
+// Host-side launchers of the MoBA kernels (internal to libmoba.so).
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace moba {
+
+cudaError_t launch_plan(const int32_t* cu_dev, int nseq, int B, int NB, const BlockTables& tb,
+                        int* counts, int ncounts, int* status, cudaStream_t stream);
+
+cudaError_t launch_centroids(const void* k, const int32_t* cu_dev, int nseq, int max_nb, int G,
+                             int d, int B, int total_nb, int num_sms, float* out,
+                             cudaStream_t stream);
+
+cudaError_t launch_gate(const void* q, const float* cents, const int32_t* cu_dev, int nseq,
+                        int max_nb, int T, int H, int G, int d, int B, int topk, int32_t* idx,
+                        cudaStream_t stream);
+
+cudaError_t launch_route_count(const int32_t* idx, const BlockTables& tb, int T, int H, int G,
+                               int topk, int NB, int b0, int nblk, int T0, int max_nb,
+                               int* counts, cudaStream_t stream);
+
+cudaError_t launch_route_scan(int* counts, int nbk, int* cursor, int4* tiles, int* n_tiles,
+                              cudaStream_t stream);
+
+cudaError_t launch_route_scatter(const int32_t* idx, const BlockTables& tb, int T, int H, int G,
+                                 int topk, int NB, int b0, int nblk, int T0, int max_nb,
+                                 int* cursor, int* entries, cudaStream_t stream);
+
+struct AttnLaunch {
+  const void* q;
+  const void* k;
+  const void* v;
+  const int4* tiles;
+  const int* n_routed;
+  const int* entries;
+  BlockTables tb;
+  void* part_o;
+  float* part_lse;
+  int* status;
+  int T, H, G, d, B, topk, NB;
+  int b0, nblk, T0;
+  float scale;
+  int grid;
+};
+
+cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream);
+
+cudaError_t launch_merge(const void* part_o, const float* part_lse, const int32_t* cu_dev,
+                         int nseq, int T, int H, int d, int B, int topk, int T0, int ntok,
+                         void* o, float* lse, cudaStream_t stream);
+
+}  // namespace moba

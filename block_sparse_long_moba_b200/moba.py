@@ -1,0 +1,187 @@
+"""Python binding of libmoba.so (ctypes): argument marshalling only.
+
+Every step of the MoBA forward pass runs in the library's CUDA kernels; PyTorch only provides
+device memory and the current stream. The functions mirror the C entry points of include/moba.h
+and raise if the library is missing or a call fails — there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoba.so")
+
+STATUS = {0: "MOBA_OK", -1: "MOBA_ERR_ARG", -2: "MOBA_ERR_UNSUPPORTED", -3: "MOBA_ERR_WORKSPACE",
+          -4: "MOBA_ERR_CUDA", -5: "MOBA_ERR_DEVICE_CHECK", -6: "MOBA_ERR_TIMEOUT"}
+KERNEL_CLASSES = ["centroid", "gate", "route_count", "route_scan", "route_scatter", "attention",
+                  "merge", "plan"]
+
+# every symbol include/moba.h declares
+EXPORTS = ["moba_status_string", "moba_version", "moba_workspace_bytes", "moba_centroids",
+           "moba_gate_topk", "moba_attn_fwd", "moba_device_status", "moba_timing_enable",
+           "moba_timing_reset", "moba_timing_read", "moba_launch_count"]
+
+
+class MobaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what} failed: {STATUS.get(status, status)}")
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmoba.so (build it with `python -m block_sparse_long_moba_b200.build`)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libmoba.so not found at {path}; build it with "
+                          "`python -m block_sparse_long_moba_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, L, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float, ctypes.c_size_t
+    lib.moba_status_string.argtypes = [I]
+    lib.moba_status_string.restype = ctypes.c_char_p
+    lib.moba_version.restype = I
+    lib.moba_workspace_bytes.argtypes = [I, P, I, I, I, I, I]
+    lib.moba_workspace_bytes.restype = S
+    lib.moba_centroids.argtypes = [P, P, P, I, I, I, I, P, P]
+    lib.moba_centroids.restype = I
+    lib.moba_gate_topk.argtypes = [P, P, P, P, I, I, I, I, I, I, P, P]
+    lib.moba_gate_topk.restype = I
+    lib.moba_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, P, P, S, P]
+    lib.moba_attn_fwd.restype = I
+    lib.moba_device_status.argtypes = [P, P]
+    lib.moba_device_status.restype = I
+    lib.moba_timing_enable.argtypes = [I]
+    lib.moba_timing_enable.restype = I
+    lib.moba_timing_reset.restype = I
+    lib.moba_timing_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(L), I]
+    lib.moba_timing_read.restype = I
+    lib.moba_launch_count.restype = L
+    _lib = lib
+    return lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise MobaError(status, what)
+
+
+def _host_cu(cu_seqlens_host) -> Tuple[ctypes.Array, int]:
+    vals = [int(x) for x in (cu_seqlens_host.tolist() if torch.is_tensor(cu_seqlens_host)
+                             else cu_seqlens_host)]
+    arr = (ctypes.c_int32 * len(vals))(*vals)
+    return arr, len(vals) - 1
+
+
+def num_blocks(cu_seqlens_host: Sequence[int], block_size: int) -> int:
+    cu = [int(x) for x in cu_seqlens_host]
+    return sum((cu[s + 1] - cu[s] + block_size - 1) // block_size for s in range(len(cu) - 1))
+
+
+def moba_workspace_bytes(cu_seqlens_host, hq: int, hkv: int, d: int, block_size: int,
+                         topk: int) -> int:
+    arr, nseq = _host_cu(cu_seqlens_host)
+    return int(load_library().moba_workspace_bytes(nseq, arr, hq, hkv, d, block_size, topk))
+
+
+def moba_centroids(k: torch.Tensor, cu_seqlens: torch.Tensor, cu_seqlens_host, block_size: int,
+                   out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Block centroids [NB, Hkv, d] fp32 of bf16 keys [T, Hkv, d]."""
+    arr, nseq = _host_cu(cu_seqlens_host)
+    T, hkv, d = k.shape
+    nb = num_blocks(list(arr), block_size)
+    if out is None:
+        out = torch.empty((nb, hkv, d), dtype=torch.float32, device=k.device)
+    st = load_library().moba_centroids(_ptr(k), _ptr(cu_seqlens), arr, nseq, hkv, d, block_size,
+                                       _ptr(out), _stream(stream))
+    _check(st, "moba_centroids")
+    return out
+
+
+def moba_gate_topk(q: torch.Tensor, centroids: torch.Tensor, cu_seqlens: torch.Tensor,
+                   cu_seqlens_host, block_size: int, topk: int,
+                   out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Routing [Hq, T, topk] int32 (ascending local block ids, -1 padded)."""
+    arr, nseq = _host_cu(cu_seqlens_host)
+    T, hq, d = q.shape
+    hkv = centroids.shape[1]
+    if out is None:
+        out = torch.empty((hq, T, topk), dtype=torch.int32, device=q.device)
+    st = load_library().moba_gate_topk(_ptr(q), _ptr(centroids), _ptr(cu_seqlens), arr, nseq, hq,
+                                       hkv, d, block_size, topk, _ptr(out), _stream(stream))
+    _check(st, "moba_gate_topk")
+    return out
+
+
+def moba_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+                  cu_seqlens_host, block_size: int, topk: int, scale: Optional[float] = None,
+                  block_idx_in: Optional[torch.Tensor] = None,
+                  block_idx_out: Optional[torch.Tensor] = None,
+                  o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None):
+    """MoBA forward: returns (o [T,Hq,d] bf16, lse [Hq,T] fp32). Buffers may be passed in."""
+    arr, nseq = _host_cu(cu_seqlens_host)
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    if scale is None:
+        scale = d ** -0.5
+    lib = load_library()
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((hq, T), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nbytes = int(lib.moba_workspace_bytes(nseq, arr, hq, hkv, d, block_size, topk))
+        if nbytes == 0 and T > 0:
+            raise MobaError(-1, "moba_workspace_bytes")
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    st = lib.moba_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), arr, nseq, hq, hkv, d,
+                           block_size, topk, ctypes.c_float(scale), _ptr(block_idx_in),
+                           _ptr(block_idx_out), _ptr(o), _ptr(lse), _ptr(workspace),
+                           ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check(st, "moba_attn_fwd")
+    return o, lse
+
+
+def moba_device_status(workspace: torch.Tensor, stream=None) -> int:
+    return int(load_library().moba_device_status(_ptr(workspace), _stream(stream)))
+
+
+def timing_enable(on: bool = True):
+    load_library().moba_timing_enable(1 if on else 0)
+
+
+def timing_reset():
+    load_library().moba_timing_reset()
+
+
+def timing_read() -> dict:
+    lib = load_library()
+    n = len(KERNEL_CLASSES)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_longlong * n)()
+    r = lib.moba_timing_read(ms, cnt, n)
+    if r < 0:
+        raise MobaError(r, "moba_timing_read")
+    return {KERNEL_CLASSES[i]: (float(ms[i]), int(cnt[i])) for i in range(n)}
+
+
+def launch_count() -> int:
+    return int(load_library().moba_launch_count())

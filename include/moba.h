@@ -1,0 +1,143 @@
+/*
+ * moba.h — C ABI of libmoba.so: the MoBA (Mixture of Block Attention) causal prefill forward
+ * pass on NVIDIA B200 (sm_100a).
+ *
+ * The method [MoBA paper summary (atlas.scime.ai), "Approach"; MoBA README (rpkg.in mirror),
+ * "Introducing MoBA"]: keys of every sequence are cut into fixed-size blocks; each block is
+ * mean-pooled into a centroid; every query head scores the PAST blocks of its sequence by
+ * q . centroid (a gate with no parameters), never a future block, always keeps its own current
+ * block and routes to the top-k blocks (the current one counted in k). Attention is exact softmax
+ * attention over the keys of the selected blocks, causal inside the current block.
+ *
+ * Conventions shared by every entry point
+ *   - Layouts (row-major, contiguous):
+ *       q            bf16  [T, Hq,  d]
+ *       k, v         bf16  [T, Hkv, d]
+ *       cu_seqlens   int32 [nseq + 1], cu[0] = 0, non-decreasing, cu[nseq] = T (packed varlen)
+ *       centroids    fp32  [NB, Hkv, d]   NB = sum_s ceil((cu[s+1]-cu[s]) / block_size)
+ *       block_idx    int32 [Hq, T, topk]  local block ids of the sequence, ascending, the
+ *                                         current block last among the valid ones, -1 padded
+ *       o            bf16  [T, Hq, d]
+ *       lse          fp32  [Hq, T]        natural-log sum-exp of the scaled logits
+ *     Global block b numbers the blocks of sequence 0, then sequence 1, ... Blocks never cross
+ *     sequence boundaries; the last block of a sequence may be short.
+ *   - Query head h reads kv head h / (Hq / Hkv) (contiguous GQA groups).
+ *   - The gate score is the unscaled dot product q . centroid in fp32; `scale` only multiplies the
+ *     attention logits.
+ *   - cu_seqlens is passed twice: on the device (read by kernels) and on the host (read to size
+ *     grids and the workspace without a device sync). Both must hold the same values.
+ *   - Memory: the caller owns every buffer (inputs, outputs and the workspace). The library never
+ *     allocates device memory. All device pointers must be 16-byte aligned.
+ *   - Streams: all work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *     Calls return after enqueueing; they never synchronise the device. Outputs are valid once
+ *     the stream reaches that point.
+ *   - Errors: every call returns a moba_status. Argument errors are detected on the host before
+ *     anything is launched. Kernels never trap: a device-side failure (a bounded wait that ran
+ *     out) is recorded in the workspace's status word; read it with moba_device_status().
+ *   - Supported shapes: d in {64, 128}; Hq % Hkv == 0; block_size a positive multiple of 64;
+ *     1 <= topk <= 64; at most 32768 blocks in one sequence; T < 2^31 / Hq.
+ *   - Device: compute capability 10.0 (B200, sm_100a); anything else gives
+ *     MOBA_ERR_UNSUPPORTED.
+ */
+#ifndef MOBA_H_
+#define MOBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOBA_OK = 0,
+  MOBA_ERR_ARG = -1,          /* invalid argument (null / misaligned pointer, bad sizes)      */
+  MOBA_ERR_UNSUPPORTED = -2,  /* valid but outside the supported shapes or device             */
+  MOBA_ERR_WORKSPACE = -3,    /* workspace smaller than moba_workspace_bytes()                */
+  MOBA_ERR_CUDA = -4,         /* a CUDA runtime / driver call or a kernel launch failed       */
+  MOBA_ERR_DEVICE_CHECK = -5, /* a device-side check failed (see moba_device_status)          */
+  MOBA_ERR_TIMEOUT = -6       /* a bounded device-side wait ran out (see moba_device_status)  */
+} moba_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moba_status_string(int status);
+
+/* Library version, (major << 16) | (minor << 8) | patch. */
+int moba_version(void);
+
+/*
+ * Bytes of device workspace moba_attn_fwd needs for this problem (0 on invalid arguments).
+ * Depends only on the host-side sizes. The workspace holds block tables, centroids, the routing
+ * (when the caller passes no block_idx_out), the inverted routing lists and the per-block partial
+ * outputs of one query chunk; chunks are sized so the partials stay under a fixed budget.
+ */
+size_t moba_workspace_bytes(int nseq, const int32_t* cu_seqlens_host, int Hq, int Hkv, int d,
+                            int block_size, int topk);
+
+/*
+ * Step 1 — block centroids [MoBA paper summary, "Approach": mean-pooled keys].
+ *   centroids[b, g, :] = (1 / n_b) * sum of k[t, g, :] over the n_b keys of global block b,
+ *   accumulated in fp32 (one pass over K with 16-byte loads).
+ * k: device bf16 [T, Hkv, d]; centroids: device fp32 [NB, Hkv, d] (written).
+ */
+int moba_centroids(const void* k, const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
+                   int nseq, int Hkv, int d, int block_size, float* centroids, void* stream);
+
+/*
+ * Step 2 — parameter-less causal top-k gate [MoBA paper summary, "Approach"; MoBA README,
+ * "Parameter-less Gating Mechanism"].
+ *   For query t in local block i of its sequence and head h (kv head g = h / (Hq/Hkv)):
+ *   s_j = q[t,h] . centroids[base + j, g] for past blocks j < i; the selection is {i} plus the
+ *   top-(topk-1) past blocks by s_j (equal scores: lower j first); if topk-1 >= i every block
+ *   0..i is selected. The T x NB score matrix is never materialised.
+ * q: device bf16 [T, Hq, d]; centroids: device fp32 [NB, Hkv, d] (e.g. from moba_centroids);
+ * block_idx: device int32 [Hq, T, topk] (written: ascending, -1 padded).
+ */
+int moba_gate_topk(const void* q, const float* centroids, const int32_t* cu_seqlens_dev,
+                   const int32_t* cu_seqlens_host, int nseq, int Hq, int Hkv, int d,
+                   int block_size, int topk, int32_t* block_idx, void* stream);
+
+/*
+ * The whole forward pass: centroids -> gate -> routing inversion -> block-sparse attention ->
+ * LSE merge [MoBA paper summary, "Approach"; FlashMoBA story: gathering scattered blocks into
+ * dense tiles].
+ *   o[t, h, :] = sum_u softmax_u(scale * q[t,h] . k[u,g]) v[u, g] over the keys u of the selected
+ *   blocks (keys <= t inside the current block); lse[h, t] = log sum_u exp(scale * q . k_u).
+ * block_idx_in : nullable. When given (device int32 [Hq, T, topk], same format as the gate's
+ *                output), this routing is used and no centroid / gate work runs. The caller
+ *                guarantees it is valid (current block present, no future block, ascending).
+ * block_idx_out: nullable. When given, receives the routing that was used.
+ * workspace    : device buffer of at least moba_workspace_bytes(...) bytes, 256-byte aligned.
+ */
+int moba_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_dev,
+                  const int32_t* cu_seqlens_host, int nseq, int Hq, int Hkv, int d,
+                  int block_size, int topk, float scale, const int32_t* block_idx_in,
+                  int32_t* block_idx_out, void* o, float* lse, void* workspace,
+                  size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then reads the status word a moba_attn_fwd call left in `workspace`:
+ * MOBA_OK, or MOBA_ERR_TIMEOUT when a bounded device wait ran out (the outputs of that call are
+ * then undefined). The word is cleared by the next moba_attn_fwd on the same workspace.
+ */
+int moba_device_status(const void* workspace, void* stream);
+
+/*
+ * Instrumentation (off by default). When enabled, every kernel launch of the library is
+ * bracketed by CUDA events recorded on the launching stream. moba_timing_read synchronises the
+ * recorded events and writes, for each kernel class, the summed device milliseconds and launch
+ * count since the last reset; kernel classes, in order: centroid, gate, route_count, route_scan,
+ * route_scatter, attention, merge, plan. Returns the number of classes (8), or a negative status.
+ */
+int moba_timing_enable(int enable);
+int moba_timing_reset(void);
+int moba_timing_read(double* ms_per_class, long long* launches_per_class, int n);
+
+/* Number of kernels this library has launched since it was loaded (all entry points). */
+long long moba_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOBA_H_ */
