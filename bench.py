@@ -1,0 +1,445 @@
+#!/usr/bin/env python
+"""Throughput of the MoBA causal prefill forward pass on B200, one process per GPU.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one full forward pass (centroids, gate, routing inversion, attention, merge) over one
+synthetic batch that is already resident in HBM. With N > 1 (launched by torchrun) every rank
+runs its own independent problem of the same shape (weak scaling: no data-path collective; the
+only collectives are the barrier and the max-over-ranks of the timed region).
+
+Prints ONE JSON line on rank 0. `--impl reference` times the fp64 CPU oracle on a bounded sample
+of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_long_moba_b200 import workloads as wl  # noqa: E402
+
+METRIC = "MoBA prefill query-tokens/s (TFLOP/s, % of bf16 tensor peak)"
+UNIT = "query-tokens/s"
+L2_BYTES = 126 * 2 ** 20
+
+
+# ----------------------------------------------------------------------------- problem sizes
+def attended_pairs(w: wl.Workload) -> int:
+    """Sum over (t, h) of the number of keys attended: (n_sel - 1) full past blocks plus the
+    causal prefix of the current block, n_sel = min(topk, i + 1). Independent of which past
+    blocks are chosen (past blocks are never a sequence's short last block)."""
+    tot = 0
+    B, k = w.block_size, w.topk
+    for s in range(w.nseq):
+        L = w.cu_seqlens[s + 1] - w.cu_seqlens[s]
+        for i in range((L + B - 1) // B):
+            n = min(B, L - i * B)
+            nsel = min(k, i + 1)
+            tot += n * (nsel - 1) * B + n * (n + 1) // 2
+    return tot * w.hq
+
+
+def useful_flops(w: wl.Workload) -> float:
+    return 4.0 * w.d * attended_pairs(w)
+
+
+def gate_flops(w: wl.Workload) -> float:
+    """2 d per scored (t, h, past block); rows with topk-1 >= i score nothing."""
+    tot = 0
+    B, k = w.block_size, w.topk
+    for s in range(w.nseq):
+        L = w.cu_seqlens[s + 1] - w.cu_seqlens[s]
+        for i in range((L + B - 1) // B):
+            if k - 1 < i and k > 1:
+                tot += min(B, L - i * B) * i
+    return 2.0 * w.d * w.hq * tot
+
+
+def kernel_bytes(w: wl.Workload) -> dict:
+    """Algorithmic HBM bytes per launch of the HBM-bound kernels (one chunk)."""
+    T, H, G, d, k = w.total_tokens, w.hq, w.hkv, w.d, w.topk
+    NB = w.num_blocks
+    routed = 0
+    B = w.block_size
+    for s in range(w.nseq):
+        L = w.cu_seqlens[s + 1] - w.cu_seqlens[s]
+        for i in range((L + B - 1) // B):
+            routed += min(B, L - i * B) * (min(k, i + 1) - 1)
+    routed *= H
+    rows = T * H  # (t, h)
+    slots = rows * 0
+    for s in range(w.nseq):
+        L = w.cu_seqlens[s + 1] - w.cu_seqlens[s]
+        for i in range((L + B - 1) // B):
+            slots += min(B, L - i * B) * min(k, i + 1)
+    slots *= H
+    return {
+        "centroid": T * G * d * 2 + NB * G * d * 4,
+        "gate": T * H * d * 2 + T * H * k * 4,
+        "route_count": T * H * k * 4,
+        "route_scatter": T * H * k * 4 + routed * 4,
+        "merge": slots * (2 * d + 4) + T * H * (2 * d + 4),
+    }
+
+
+# ------------------------------------------------------------------------------------ peaks
+def read_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"]),
+                "bf16_tflops_sustained": float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            self.path = f"/tmp/moba_clocks_{os.getpid()}.csv"
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# -------------------------------------------------------------------------------- CPU oracle
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample_rate(w: wl.Workload, q, k, v, target_s: float = 15.0, seed: int = 0) -> dict:
+    """Time the fp64 oracle (as it stands) on a bounded sample of query tokens (all heads):
+    centroids of the whole K (charged pro rata to the sample), gate and attention of the sample.
+    Returns query-tokens/s."""
+    from oracle import moba_ref as ref
+
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+    t0 = time.perf_counter()
+    cents = ref.centroids(kc, w.cu_seqlens, w.block_size)
+    t_cent = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    T = w.total_tokens
+    done_tok, t_rows, n = 0, 0.0, 4
+    while t_rows < target_s and done_tok < T:
+        toks = np.sort(rng.choice(T, size=min(n, T), replace=False))
+        t1 = time.perf_counter()
+        rt = ref.select_blocks(qc, cents, w.cu_seqlens, w.block_size, w.topk, toks)
+        ref.attention(qc, kc, vc, w.cu_seqlens, w.block_size, rt.idx, w.scale, toks)
+        t_rows += time.perf_counter() - t1
+        done_tok += len(toks)
+        n = min(n * 2, 4096)
+    charged = t_rows + t_cent * done_tok / T
+    return {"value": done_tok / charged, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{done_tok} random query tokens x all {w.hq} heads of {w.name} "
+                      f"(gate + attention {t_rows:.1f} s) + centroids of all {w.num_blocks} blocks "
+                      f"({t_cent:.1f} s, charged pro rata {done_tok}/{T})"}
+
+
+# ------------------------------------------------------------------------------- distributed
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def physical_gpu_index(local: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local < len(ids) and ids[local].isdigit():
+            return int(ids[local])
+    return local
+
+
+# ----------------------------------------------------------------------------------- our arm
+def run_ours(args):
+    from block_sparse_long_moba_b200 import build, moba
+
+    world, rank, local = dist_setup(args.gpus)
+    if rank == 0:
+        build.build()
+    barrier(world)
+    moba.load_library()
+    w = wl.WORKLOADS[args.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v, cu = wl.make_inputs(w, seed=rank, device=dev)
+    T, H, d = w.total_tokens, w.hq, w.d
+    o = torch.empty_like(q)
+    lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+    idx = torch.empty((H, T, w.topk), dtype=torch.int32, device=dev)
+    ws = torch.empty(moba.moba_workspace_bytes(w.cu_seqlens, H, w.hkv, d, w.block_size, w.topk),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        moba.moba_attn_fwd(q, k, v, cu, w.cu_seqlens, w.block_size, w.topk, w.scale,
+                           block_idx_out=idx, o=o, lse=lse, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = moba.moba_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+
+    # ---- device-timed region: inputs resident in HBM
+    moba.timing_reset()
+    moba.timing_enable(True)
+    clocks = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    n0 = moba.launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = moba.launch_count() - n0
+    clk = clocks.stop() if clocks else None
+    moba.timing_enable(False)
+    per_kernel = moba.timing_read()
+    ms_local = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms_local, world)
+    status = moba.moba_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    # ---- end to end through the public API: pinned host inputs -> device -> host outputs
+    qh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True).copy_(q)
+    kh = torch.empty(k.shape, dtype=k.dtype, pin_memory=True).copy_(k)
+    vh = torch.empty(v.shape, dtype=v.dtype, pin_memory=True).copy_(v)
+    cuh = torch.tensor(w.cu_seqlens, dtype=torch.int32).pin_memory()
+    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh, cuh))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+
+    def e2e_step():
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        cu.copy_(cuh, non_blocking=True)
+        moba.moba_attn_fwd(q, k, v, cu, w.cu_seqlens, w.block_size, w.topk, w.scale, o=o,
+                           lse=lse, workspace=ws, stream=stream)
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world) / e2e_steps
+
+    if rank == 0:
+        peaks = read_peaks()
+        ms_step = ms / args.steps
+        value = world * T / (ms_step / 1e3)
+        uf = useful_flops(w)
+        attn_ms, attn_n = per_kernel["attention"]
+        attn_avg = attn_ms / max(attn_n, 1)
+        launches_per_step = max(attn_n // args.steps, 1)
+        achieved = uf / launches_per_step / (attn_avg / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        kb = kernel_bytes(w)
+        kern = {}
+        for name, (kms, kn) in per_kernel.items():
+            if kn == 0:
+                continue
+            ent = {"ms_per_launch": kms / kn, "launches": kn, "share": kms / max(ms_local, 1e-9)}
+            if name in kb:
+                gbs = kb[name] / (kms / kn / 1e3) / 1e9 / (1 if name != "merge" else 1)
+                ent["gbs"] = gbs
+                ent["hbm_frac"] = gbs / peaks["hbm_gbs"]
+            kern[name] = ent
+        if "gate" in kern:
+            kern["gate"]["gate_tflops_fp32"] = gate_flops(w) / (kern["gate"]["ms_per_launch"] / 1e3) / 1e12
+        traffic = None
+        tpath = os.path.join(ROOT, "profiles", f"attention_{w.name}_traffic.json")
+        if os.path.exists(tpath):
+            try:
+                with open(tpath) as f:
+                    traffic = json.load(f).get("bytes_per_launch")
+            except Exception:
+                traffic = None
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; Q,V ~ N(0,1), K = N(0,1) + per-block offset)",
+            "config": {"workload": w.name, "T": T, "hq": H, "hkv": w.hkv, "d": d,
+                       "block_size": w.block_size, "topk": w.topk, "nseq": w.nseq,
+                       "parallelism": f"independent problem per GPU x{world}",
+                       "l2": "no flush: Q/K/V inputs are larger than L2"},
+            "tflops_useful": uf * world / (ms_step / 1e3) / 1e12,
+            "tflops_frac_of_peak_sustained": uf / (ms_step / 1e3) / 1e12 / peak,
+            "roofline": {"kernel": "attention", "bound": "tensor", "achieved": achieved,
+                         "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_kind": f"bf16 dense sustained, {peaks['source']}",
+                         "frac_of_burst": achieved / peaks["bf16_tflops"],
+                         "traffic": traffic},
+            "kernels": kern,
+            "gpu_launches": launches,
+            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_sample_rate(w, q, k, v, target_s=args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = wl.WORKLOADS[args.workload]
+    q, k, v, cu = wl.make_inputs(w, seed=0, device="cpu")
+    for _ in range(args.warmup):
+        oracle_sample_rate(w, q, k, v, target_s=min(2.0, args.cpu_seconds))
+    vals = []
+    t0 = time.perf_counter()
+    last = None
+    for _ in range(args.steps):
+        last = oracle_sample_rate(w, q, k, v, target_s=args.cpu_seconds / max(args.steps, 1))
+        vals.append(last["value"])
+    wall = time.perf_counter() - t0
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": wall * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "T": w.total_tokens, "hq": w.hq, "hkv": w.hkv, "d": w.d,
+                   "block_size": w.block_size, "topk": w.topk},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": last["sample"] if last else ""},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama8b_128k", choices=list(wl.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
