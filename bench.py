@@ -94,6 +94,12 @@ def kernel_bytes(w: wl.Workload) -> dict:
     }
 
 
+def job_throughput(world: int, tokens_per_rank: int, ms_step_max: float) -> float:
+    """Whole-job query tokens/s: every rank processes its own problem (weak scaling), timed as
+    the max over ranks."""
+    return world * tokens_per_rank / (ms_step_max / 1e3)
+
+
 # ------------------------------------------------------------------------------------ peaks
 def read_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -224,11 +230,12 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world) -> float:
+def max_over_ranks(x: float, world, device="cuda") -> float:
+    """Max of a per-rank timing over all ranks (the job is as slow as its slowest rank)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -334,7 +341,7 @@ def run_ours(args):
     if rank == 0:
         peaks = read_peaks()
         ms_step = ms / args.steps
-        value = world * T / (ms_step / 1e3)
+        value = job_throughput(world, T, ms_step)
         uf = useful_flops(w)
         attn_ms, attn_n = per_kernel["attention"]
         attn_avg = attn_ms / max(attn_n, 1)

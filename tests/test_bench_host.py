@@ -1,0 +1,76 @@
+"""Host-side logic of bench.py (no GPU): FLOP accounting against the oracle's routing, and the
+multi-rank timing reduction with 2 gloo ranks on the CPU."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+from block_sparse_long_moba_b200 import workloads as wl
+from oracle import moba_ref as ref
+
+
+@pytest.mark.parametrize("cu,B,topk", [([0, 1000], 128, 3), ([0, 300, 300, 1111], 64, 5),
+                                       ([0, 4096], 256, 64)])
+def test_attended_pairs_match_oracle_routing(cu, B, topk):
+    w = wl.custom(cu, 2, 1, 16, B, topk)
+    q, k, v, _ = wl.make_inputs(w, device="cpu")
+    rt = ref.select_blocks(q, ref.centroids(k, cu, B), cu, B, topk)
+    bt = ref.block_table(cu, B)
+    s_of, i_of = ref.token_position(cu, B, np.arange(cu[-1]))
+    pairs = 0
+    for h in range(2):
+        for t in range(cu[-1]):
+            base = int(bt.blk_off[s_of[t]])
+            for j in rt.idx[h, t]:
+                if j >= 0:
+                    b = base + int(j)
+                    pairs += min(int(bt.end[b]), t + 1) - int(bt.start[b])
+    assert bench.attended_pairs(w) == pairs
+
+
+def test_workload_flops_of_the_headline_configs():
+    assert abs(bench.useful_flops(wl.WORKLOADS["llama8b_128k"]) / 1e12 - 83.01) < 0.01
+    assert abs(bench.useful_flops(wl.WORKLOADS["llama8b_1m"]) / 1e12 - 791.1) < 0.1
+
+
+def test_job_throughput_is_weak_scaling():
+    assert bench.job_throughput(1, 131072, 100.0) == pytest.approx(1.31072e6)
+    assert bench.job_throughput(4, 131072, 100.0) == pytest.approx(4 * 1.31072e6)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _rank_main(rank, world, port, out):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    mine = 10.0 + 5.0 * rank
+    got = bench.max_over_ranks(mine, world, device="cpu")
+    out[rank] = got
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    assert out[0] == 15.0 and out[1] == 15.0
