@@ -103,7 +103,8 @@ int check_shape(int Hq, int Hkv, int d, int B, int topk) {
   return MOBA_OK;
 }
 
-int make_plan(int nseq, const int32_t* cu, int Hq, int Hkv, int d, int B, int topk, Plan* P) {
+int make_plan(int nseq, const int32_t* cu, int Hq, int Hkv, int d, int B, int topk, Plan* P,
+              size_t partial_budget = kPartialBudgetBytes) {
   P->T = cu[nseq];
   P->blk_len.clear();
   for (int s = 0; s < nseq; ++s) {
@@ -118,7 +119,7 @@ int make_plan(int nseq, const int32_t* cu, int Hq, int Hkv, int d, int B, int to
   if (P->max_nb > 65535) return MOBA_ERR_UNSUPPORTED;
   // query chunks of whole blocks, so that partial rows (t, h, slot) fit the budget
   const size_t row_bytes = static_cast<size_t>(d) * 2 + 4 + 4;
-  size_t max_rows = kPartialBudgetBytes / row_bytes;
+  size_t max_rows = std::max<size_t>(partial_budget / row_bytes, 1);
   const size_t per_tok = static_cast<size_t>(Hq) * topk;
   max_rows = std::min<size_t>(max_rows, (1ull << 31) - 1);
   P->chunks.clear();
@@ -251,16 +252,23 @@ int moba_gate_topk(const void* q, const float* centroids, const int32_t* cu_dev,
   return MOBA_OK;
 }
 
-int moba_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_dev,
+}  // extern "C"
+
+namespace moba {
+
+// Body of moba_attn_fwd; `partial_budget` bounds the partial outputs of one query chunk.
+int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu_dev,
                   const int32_t* cu_host, int nseq, int Hq, int Hkv, int d, int block_size,
                   int topk, float scale, const int32_t* block_idx_in, int32_t* block_idx_out,
-                  void* o, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+                  void* o, float* lse, void* workspace, size_t workspace_bytes, void* stream,
+                  size_t partial_budget) {
   int st = check_cu(nseq, cu_host);
   if (st != MOBA_OK) return st;
   if ((st = check_shape(Hq, Hkv, d, block_size, topk)) != MOBA_OK) return st;
   if (!(scale > 0.f) || scale > 1e30f) return MOBA_ERR_ARG;
   Plan P;
-  if ((st = make_plan(nseq, cu_host, Hq, Hkv, d, block_size, topk, &P)) != MOBA_OK) return st;
+  if ((st = make_plan(nseq, cu_host, Hq, Hkv, d, block_size, topk, &P, partial_budget)) != MOBA_OK)
+    return st;
   if (P.T == 0) return MOBA_OK;
   if (!q || !k || !v || !cu_dev || !o || !lse || !workspace) return MOBA_ERR_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
@@ -330,6 +338,29 @@ int moba_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu
                              c.ntok, o, lse, s));
   }
   return MOBA_OK;
+}
+
+size_t workspace_bytes_for(int nseq, const int32_t* cu_host, int Hq, int Hkv, int d,
+                           int block_size, int topk, size_t partial_budget) {
+  if (check_cu(nseq, cu_host) != MOBA_OK) return 0;
+  if (check_shape(Hq, Hkv, d, block_size, topk) != MOBA_OK) return 0;
+  Plan P;
+  if (make_plan(nseq, cu_host, Hq, Hkv, d, block_size, topk, &P, partial_budget) != MOBA_OK)
+    return 0;
+  return layout_of(P, nseq, Hq, Hkv, d, topk).total;
+}
+
+}  // namespace moba
+
+extern "C" {
+
+int moba_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_dev,
+                  const int32_t* cu_host, int nseq, int Hq, int Hkv, int d, int block_size,
+                  int topk, float scale, const int32_t* block_idx_in, int32_t* block_idx_out,
+                  void* o, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  return attn_fwd_impl(q, k, v, cu_dev, cu_host, nseq, Hq, Hkv, d, block_size, topk, scale,
+                       block_idx_in, block_idx_out, o, lse, workspace, workspace_bytes, stream,
+                       kPartialBudgetBytes);
 }
 
 int moba_device_status(const void* workspace, void* stream) {

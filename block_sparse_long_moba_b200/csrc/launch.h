@@ -52,4 +52,16 @@ cudaError_t launch_merge(const void* part_o, const float* part_lse, const int32_
                          int nseq, int T, int H, int d, int B, int topk, int T0, int ntok,
                          void* o, float* lse, cudaStream_t stream);
 
+// Whole forward pass on a caller-provided workspace (the body of moba_attn_fwd); the partial
+// outputs of one query chunk are kept under `partial_budget` bytes.
+int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu_dev,
+                  const int32_t* cu_host, int nseq, int Hq, int Hkv, int d, int block_size,
+                  int topk, float scale, const int32_t* block_idx_in, int32_t* block_idx_out,
+                  void* o, float* lse, void* workspace, size_t workspace_bytes, void* stream,
+                  size_t partial_budget);
+
+// Workspace bytes attn_fwd_impl needs with the given chunk budget (0 on invalid arguments).
+size_t workspace_bytes_for(int nseq, const int32_t* cu_host, int Hq, int Hkv, int d,
+                           int block_size, int topk, size_t partial_budget);
+
 }  // namespace moba

@@ -23,7 +23,10 @@ KERNEL_CLASSES = ["centroid", "gate", "route_count", "route_scan", "route_scatte
 # every symbol include/moba.h declares
 EXPORTS = ["moba_status_string", "moba_version", "moba_workspace_bytes", "moba_centroids",
            "moba_gate_topk", "moba_attn_fwd", "moba_device_status", "moba_timing_enable",
-           "moba_timing_reset", "moba_timing_read", "moba_launch_count"]
+           "moba_timing_reset", "moba_timing_read", "moba_launch_count",
+           "moba_attn_fwd_noalloc"]
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class MobaError(RuntimeError):
@@ -64,6 +67,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moba_timing_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(L), I]
     lib.moba_timing_read.restype = I
     lib.moba_launch_count.restype = L
+    lib.moba_attn_fwd_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P, P, P]
+    lib.moba_attn_fwd_noalloc.restype = I
     _lib = lib
     return lib
 
@@ -157,6 +162,30 @@ def moba_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens:
                            _ptr(block_idx_out), _ptr(o), _ptr(lse), _ptr(workspace),
                            ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check(st, "moba_attn_fwd")
+    return o, lse
+
+
+def moba_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                          cu_seqlens: torch.Tensor, cu_seqlens_host, block_size: int, topk: int,
+                          scale: Optional[float] = None, o: Optional[torch.Tensor] = None,
+                          lse: Optional[torch.Tensor] = None, stream=None):
+    """moba_attn_fwd without a workspace: the library's static scratch array is used instead
+    (for callers that cannot allocate device memory; see include/moba.h). The outputs may be
+    passed in so that the call itself allocates nothing."""
+    arr, nseq = _host_cu(cu_seqlens_host)
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    if scale is None:
+        scale = d ** -0.5
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((hq, T), dtype=torch.float32, device=q.device)
+    st = load_library().moba_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), arr,
+                                              nseq, hq, hkv, d, block_size, topk,
+                                              ctypes.c_float(scale), _ptr(o), _ptr(lse),
+                                              _stream(stream))
+    _check(st, "moba_attn_fwd_noalloc")
     return o, lse
 
 

@@ -116,6 +116,33 @@ int moba_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu
                   size_t workspace_bytes, void* stream);
 
 /*
+ * moba_attn_fwd for callers that cannot allocate device memory. The paper has no counterpart:
+ * this is a deployment variant of the same computation.
+ *
+ * Some callers may not call cudaMalloc: plug-in code whose host application owns all device
+ * memory through its own allocator or a fixed pool, and latency-critical paths that cannot
+ * afford the implicit synchronisation an allocation may cause. This entry point allocates
+ * nothing: its scratch memory is one static device array inside libmoba.so of
+ * MOBA_NOALLOC_SCRATCH_BYTES, reserved on every GPU that loads the library until the process
+ * exits. Arguments and results are those of moba_attn_fwd without routing in/out and workspace.
+ *   - Returns MOBA_ERR_WORKSPACE, launching nothing, when the problem needs more scratch than the
+ *     array holds (the routing [Hq, T, topk] int32 plus block tables, centroids and the chunked
+ *     routing lists and partial outputs; partial outputs are chunked to a quarter of the array).
+ *   - All calls share the array and it keeps the previous call's contents; each call clears what
+ *     must start at zero on its own stream. Calls that overlap on the GPU race on the array and
+ *     must be serialised by the caller.
+ *   - The first call on a device looks up the array's device address (with that device
+ *     current); make that first call before any stream capture begins.
+ *   - Device-side status (bounded waits) is not readable through moba_device_status for this
+ *     entry point; a failed wait leaves the outputs undefined.
+ */
+#define MOBA_NOALLOC_SCRATCH_BYTES (64u << 20)
+int moba_attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                          const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host, int nseq,
+                          int Hq, int Hkv, int d, int block_size, int topk, float scale, void* o,
+                          float* lse, void* stream);
+
+/*
  * Synchronises `stream`, then reads the status word a moba_attn_fwd call left in `workspace`:
  * MOBA_OK, or MOBA_ERR_TIMEOUT when a bounded device wait ran out (the outputs of that call are
  * then undefined). The word is cleared by the next moba_attn_fwd on the same workspace.
