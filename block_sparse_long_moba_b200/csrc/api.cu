@@ -140,7 +140,7 @@ int make_plan(int nseq, const int32_t* cu, int Hq, int Hkv, int d, int B, int to
     const size_t ent = static_cast<size_t>(c.ntok) * Hq * (topk - 1);
     P->max_rows = std::max(P->max_rows, rows);
     P->max_entries = std::max(P->max_entries, ent);
-    P->max_tiles = std::max(P->max_tiles, ent / kTile + static_cast<size_t>(Hkv) * P->NB + 1);
+    P->max_tiles = std::max(P->max_tiles, ent / kItemRows + static_cast<size_t>(Hkv) * P->NB + 1);
   }
   return MOBA_OK;
 }
@@ -329,8 +329,8 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu
     A.part_o = part_o; A.part_lse = part_lse; A.status = status;
     A.T = P.T; A.H = Hq; A.G = Hkv; A.d = d; A.B = block_size; A.topk = topk; A.NB = P.NB;
     A.b0 = c.b0; A.nblk = c.nblk; A.T0 = c.T0; A.scale = scale;
-    const long long P128 = (block_size + kTile - 1) / kTile;
-    const long long items = static_cast<long long>(P.max_tiles) + P128 * c.nblk * Hq;
+    const long long P256 = (block_size + kItemRows - 1) / kItemRows;
+    const long long items = static_cast<long long>(P.max_tiles) + P256 * c.nblk * Hq;
     A.grid = static_cast<int>(std::min<long long>(sms, items));
     MOBA_LAUNCH(kAttn, s, launch_attention(A, s));
     MOBA_LAUNCH(kMerge, s,

@@ -1,39 +1,45 @@
 // K4 — block-sparse attention on the tcgen05 tensor cores.
 //
-// Work items (one 128-row query tile each, processed by a persistent CTA per SM):
-//   routed tile : up to 128 (t, h) rows of one kv head g that routed to one past block b (a list
-//                 built by the routing inversion), attending every key of b — the scattered query
-//                 rows are gathered into one dense operand [FlashMoBA story, Gather-and-Densify];
-//   diagonal tile: 128 consecutive tokens of one query head inside their own block, attending the
-//                 block's keys up to the query position (causal inside the current block)
-//                 [MoBA paper summary (atlas.scime.ai), "Approach"].
+// Work items (256 query rows each, processed by persistent CTAs, one per SM):
+//   routed item  : up to 256 (t, h) rows of one kv head g that routed to one past block b (a list
+//                  built by the routing inversion), attending every key of b — the scattered query
+//                  rows are gathered into one dense operand [FlashMoBA story, Gather-and-Densify];
+//   diagonal item: 256 consecutive tokens of one query head inside their own block, attending the
+//                  block's keys up to each query's position (causal inside the current block)
+//                  [MoBA paper summary (atlas.scime.ai), "Approach"].
 // Each row's result is a normalised partial O_s (bf16) plus its log-sum-exp (fp32), written to the
 // row's slot; the merge kernel combines the slots.
 //
-// Per item, for every 128-key sub-tile j of the key range:
-//   S_j = Q K_j^T           tcgen05.mma kind::f16, A = Q (smem, K-major SW128), B = K_j (smem,
-//                           K-major SW128, loaded by TMA), fp32 accumulator in TMEM
-//   P_j = exp2(S_j * scale * log2e - m)   one thread per row (TMEM lane), written back to TMEM
-//                                         as bf16 over the S columns
-//   O  += P_j V_j           tcgen05.mma with A = P read from TMEM, B = V_j (smem, MN-major SW128)
-// The running max m is only raised when a row's max grows by more than 2^8 (then O and l are
-// rescaled), which keeps every p <= 256 and makes rescaling rare; O / l is exact either way.
+// An item is two 128-row halves A and B that share every K/V sub-tile. For each 128-key sub-tile:
+//   S_x = Q_x K^T        tcgen05.mma kind::f16, M=128 N=128, Q and K K-major (128-byte swizzle),
+//                        fp32 accumulator in TMEM
+//   P_x = exp2(S_x * scale * log2e - m)   one softmax warpgroup per half, thread = row = TMEM
+//                                         lane; P written back over S in TMEM as packed bf16
+//   O_x += P_x V         tcgen05.mma with A = P from TMEM and B = V (MN-major) from shared memory
+// The MMA issue order S_A(j), PV_B(j-1), S_B(j), PV_A(j) lets one half's softmax overlap the other
+// half's matrix products, so the tensor pipe waits on neither softmax alone. The reference max m of
+// a row is raised only when the row max grows by more than 2^8 (O and l are then rescaled in
+// TMEM); p <= 256 always, and O / l is exact either way. Because PV_x(j-1) is issued before
+// S_x(j), the arrival of S_x(j) implies O_x is complete, so a rescale never waits.
 //
-// Warp roles (256 threads): warp 0 = TMA producer of K/V sub-tiles; warp 1 = TMEM owner and MMA
-// issuer; warps 2-3 = Q row gather (cp.async into the swizzled layout); warps 4-7 = softmax and
-// epilogue (thread i <-> TMEM lane i <-> query row i). Buffers: Q x2, K x NST, V x NST in shared
-// memory; S/P x2 and O x2 in TMEM (512 columns). Every wait is bounded (2 s); on a timeout the
-// kernel raises a CTA abort flag, records a status code and every role leaves its loop.
+// Warp roles (384 threads): warp 0 = TMA producer of K/V sub-tiles; warp 1 = TMEM owner and MMA
+// issuer (both run converged and let elect.sync pick the issuing lane); warps 2-3 = Q row gather (cp.async into the swizzled layout); warps 4-7 = softmax and
+// epilogue of half A; warps 8-11 = the same for half B. Every wait is bounded (2 s); on a timeout
+// the kernel raises a CTA abort flag, records a status code, drains what it has in flight and
+// returns.
 #include "common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
 
 namespace moba {
 
+// Column pairs (of every 8) whose exp2 runs on the FMA pipe instead of MUFU.EX2, balancing the two.
+constexpr int kPolyPairs = 0;
+
 struct AttnArgs {
   const __nv_bfloat16* q;  // [T, H, D]
-  const int4* tiles;       // routed tiles: {bucket, first entry, rows, -}
-  const int* n_routed;     // device count of routed tiles
+  const int4* tiles;       // routed items: {bucket, first entry, rows, -}
+  const int* n_routed;     // device count of routed items
   const int* entries;      // partial row of every routed (t, h, slot)
   BlockTables tb;
   __nv_bfloat16* part_o;   // [rows, D]
@@ -41,8 +47,8 @@ struct AttnArgs {
   int* status;
   int T, H, G, r, topk, NB;
   int b0, nblk, T0;        // chunk: global blocks [b0, b0 + nblk), first token T0
-  int P;                   // ceil(B / 128): 128-row tiles per block
-  int n_diag;              // P * nblk * H diagonal items (some may be empty)
+  int P2;                  // ceil(B / 256): diagonal items per (block, head)
+  int n_diag;              // P2 * nblk * H diagonal items (some may be empty)
   float scale_log2;        // scale * log2(e)
 };
 
@@ -50,45 +56,49 @@ struct Item {
   int kind;  // 0 empty, 1 routed, 2 diagonal
   int g, h, b;
   int key0, klen, nsub;
-  int rows, start;       // routed: rows and first entry; diagonal: rows
-  int qtok0, p, slot;    // diagonal: first query token, tile position in block, output slot
+  int rows;     // valid rows of the item (<= 256)
+  int start;    // routed: first entry of the item
+  int qtok0;    // diagonal: first query token
+  int qoff;     // diagonal: position of the first query inside its block
+  int slot;     // diagonal: output slot of the current block
 };
 
 __device__ __forceinline__ Item decode_item(const AttnArgs& a, int w, int n_routed) {
   Item it;
   it.kind = 0;
+  it.h = 0;
+  it.start = 0;
+  it.qtok0 = 0;
+  it.qoff = 0;
+  it.slot = 0;
   if (w < n_routed) {
     const int4 tl = a.tiles[w];
     it.kind = 1;
     it.g = tl.x / a.NB;
     it.b = tl.x % a.NB;
-    it.h = 0;
     it.start = tl.y;
     it.rows = tl.z;
     it.key0 = a.tb.blk_start[it.b];
     it.klen = a.tb.blk_len[it.b];
     it.nsub = (it.klen + kTile - 1) / kTile;
-    it.qtok0 = 0;
-    it.p = 0;
-    it.slot = 0;
     return it;
   }
   const int wd = w - n_routed;
   it.h = wd % a.H;
   const int rest = wd / a.H;
   const int bl = rest % a.nblk;
-  it.p = a.P - 1 - rest / a.nblk;  // longest diagonal tiles first
+  const int p2 = a.P2 - 1 - rest / a.nblk;  // longest diagonal items first
   it.b = a.b0 + bl;
   const int len = a.tb.blk_len[it.b];
-  if (it.p * kTile >= len) return it;  // empty (short last block)
+  if (p2 * kItemRows >= len) return it;  // empty (short block)
   it.kind = 2;
   it.g = it.h / a.r;
   it.key0 = a.tb.blk_start[it.b];
-  it.klen = min(len, kTile * (it.p + 1));
-  it.nsub = it.p + 1;
-  it.rows = min(kTile, len - kTile * it.p);
-  it.start = 0;
-  it.qtok0 = it.key0 + kTile * it.p;
+  it.qoff = p2 * kItemRows;
+  it.rows = min(kItemRows, len - it.qoff);
+  it.klen = it.qoff + it.rows;  // keys up to the last query of the item
+  it.nsub = (it.klen + kTile - 1) / kTile;
+  it.qtok0 = it.key0 + it.qoff;
   const int i = it.b - a.tb.blk_off[a.tb.blk_seq[it.b]];
   it.slot = min(a.topk, i + 1) - 1;
   return it;
@@ -96,37 +106,43 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, int w, int n_rout
 
 template <int D>
 struct AttnCfg {
-  static constexpr int NCB = D / 64;                 // 64-column (128-byte) swizzle blocks
-  static constexpr int TILE_BYTES = kTile * D * 2;   // one 128 x D bf16 tile
-  static constexpr int NST = (D == 128) ? 2 : 4;     // K and V ring depth
-  static constexpr int SMEM_TILES = (2 + 2 * NST) * TILE_BYTES;
+  static constexpr int NCB = D / 64;                  // 64-column (128-byte) swizzle blocks
+  static constexpr int HALF_BYTES = kTile * D * 2;    // one 128 x D bf16 tile
+  static constexpr int Q_BYTES = 2 * HALF_BYTES;      // one 256-row item
+  static constexpr int QB = (D == 128) ? 1 : 2;       // Q buffers
+  static constexpr int NST = (D == 128) ? 2 : 4;      // K and V ring depth
+  static constexpr int SMEM_TILES = QB * Q_BYTES + 2 * NST * HALF_BYTES;
   static constexpr int SMEM_BYTES = SMEM_TILES + 1024 /*barriers*/ + 1024 /*alignment slack*/;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
+  // Registers per thread: launch budget (384 threads at 168) re-split between the control
+  // warpgroup (producer, MMA, gather) and the two softmax warpgroups; 128*72 + 256*216 = 384*168.
+  static constexpr uint32_t REGS_LAUNCH = 168, REGS_CTRL = 72, REGS_SOFTMAX = 216;
+  // TMEM columns: S/P of half x at 128 * x, O of half x at 256 + D * x
+  __host__ __device__ static constexpr uint32_t tm_s(int x) { return 128u * x; }
+  __host__ __device__ static constexpr uint32_t tm_o(int x) { return 256u + D * x; }
 };
 
 struct AttnBars {
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full[2], p_full[2];
-  uint64_t o_done, o_full[2], o_free[2];
+  uint64_t s_full[2], p_full[2], o_full[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
 
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                 const AttnArgs a) {
   using C = AttnCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;                              // [2][NCB][16 KB]
-  uint8_t* sK = sQ + 2 * C::TILE_BYTES;            // [NST][NCB][16 KB]
-  uint8_t* sV = sK + C::NST * C::TILE_BYTES;       // [NST][NCB][16 KB]
-  AttnBars* bars = reinterpret_cast<AttnBars*>(sV + C::NST * C::TILE_BYTES);
+  uint8_t* sQ = smem;                              // [QB][2 halves][NCB][16 KB]
+  uint8_t* sK = sQ + C::QB * C::Q_BYTES;           // [NST][NCB][16 KB]
+  uint8_t* sV = sK + C::NST * C::HALF_BYTES;       // [NST][NCB][16 KB]
+  AttnBars* bars = reinterpret_cast<AttnBars*>(sV + C::NST * C::HALF_BYTES);
   volatile int* abort_flag = &bars->abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -137,7 +153,6 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(&bars->s_full[x], 1);
       mbar_init(&bars->p_full[x], 128);
       mbar_init(&bars->o_full[x], 1);
-      mbar_init(&bars->o_free[x], 128);
     }
     for (int x = 0; x < C::NST; ++x) {
       mbar_init(&bars->k_full[x], 1);
@@ -145,7 +160,6 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(&bars->v_full[x], 1);
       mbar_init(&bars->v_empty[x], 1);
     }
-    mbar_init(&bars->o_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -168,33 +182,38 @@ __global__ void __launch_bounds__(256, 1)
   const uint64_t TO = kWaitTimeoutNs;
   int* err = a.status;
 
-  if (warp == 0) {
+  if (warp < 4) {
+   regs_dec<C::REGS_CTRL>();
+   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer (K, V)
-    if (lane == 0) {
+    // The whole warp runs the loop (converged); elect.sync picks the issuing lane.
+    {
       uint32_t J = 0, issued_k = 0, issued_v = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
         const Item it = decode_item(a, w, n_routed);
         if (it.kind == 0) continue;
-        for (int j = 0; j < it.nsub && ok; ++j, ++J) {
+        for (int j = 0; j < it.nsub; ++j, ++J) {
           const int st = J % C::NST;
           const uint32_t ph = (J / C::NST) & 1;
           const int tok = it.key0 + j * kTile;
-          ok = mbar_wait_bounded(&bars->k_empty[st], ph ^ 1, abort_flag, err, kDevTimeoutAttn, TO);
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->k_empty[st], ph ^ 1, abort_flag,
+                                                         err, kDevTimeoutAttn, TO));
           if (!ok) break;
-          mbar_arrive_expect_tx(&bars->k_full[st], C::TILE_BYTES);
+          mbar_arrive_expect_tx_elect(&bars->k_full[st], C::HALF_BYTES);
 #pragma unroll
           for (int c = 0; c < C::NCB; ++c)
-            tma_load_3d(sK + st * C::TILE_BYTES + c * 16384, &map_k, &bars->k_full[st], c * 64,
-                        it.g, tok);
+            tma_load_3d_elect(sK + st * C::HALF_BYTES + c * 16384, &map_k, &bars->k_full[st],
+                              c * 64, it.g, tok);
           ++issued_k;
-          ok = mbar_wait_bounded(&bars->v_empty[st], ph ^ 1, abort_flag, err, kDevTimeoutAttn, TO);
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->v_empty[st], ph ^ 1, abort_flag,
+                                                         err, kDevTimeoutAttn, TO));
           if (!ok) break;
-          mbar_arrive_expect_tx(&bars->v_full[st], C::TILE_BYTES);
+          mbar_arrive_expect_tx_elect(&bars->v_full[st], C::HALF_BYTES);
 #pragma unroll
           for (int c = 0; c < C::NCB; ++c)
-            tma_load_3d(sV + st * C::TILE_BYTES + c * 16384, &map_v, &bars->v_full[st], c * 64,
-                        it.g, tok);
+            tma_load_3d_elect(sV + st * C::HALF_BYTES + c * 16384, &map_v, &bars->v_full[st],
+                              c * 64, it.g, tok);
           ++issued_v;
         }
       }
@@ -215,82 +234,90 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop (converged, warp-uniform descriptors); elect.sync picks the
+    // lane that issues each tcgen05.mma / commit.
+    {
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       uint32_t J = 0, lt = 0;
       bool ok = true;
-      // the PV of sub-tile J-1 is issued after the QK of sub-tile J (software pipelining)
-      bool pend = false;
-      uint32_t pend_J = 0, pend_ob = 0, pend_lt = 0;
-      bool pend_first = false, pend_last = false;
-      auto issue_pv = [&](uint32_t Jp, uint32_t ob, uint32_t ltp, bool first, bool last) -> bool {
-        const uint32_t sb = Jp & 1;
+      auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu,
+                          mbar_wait_bounded(bar, parity, abort_flag, err, kDevTimeoutAttn, TO));
+      };
+      auto issue_s = [&](int half, uint32_t qb, int st) {
+        const uint32_t t_s = tmem + C::tm_s(half);
+        const uint32_t qbase = sQa + qb * C::Q_BYTES + half * C::HALF_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          const uint64_t ad = smem_desc_sw128(qbase + off, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sKa + st * C::HALF_BYTES + off, 16, 1024);
+          mma_ss_elect(t_s, ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
+        }
+        mma_commit_elect(&bars->s_full[half]);
+      };
+      // O_x += P_x V_st; waits for P_x of sub-tile Jp
+      auto issue_pv = [&](int half, uint32_t Jp, bool first, bool last) -> bool {
         const int st = Jp % C::NST;
-        if (!mbar_wait_bounded(&bars->p_full[sb], (Jp >> 1) & 1, abort_flag, err, kDevTimeoutAttn, TO))
-          return false;
-        if (!mbar_wait_bounded(&bars->v_full[st], (Jp / C::NST) & 1, abort_flag, err, kDevTimeoutAttn, TO))
-          return false;
-        if (first && !mbar_wait_bounded(&bars->o_free[ob], ((ltp >> 1) & 1) ^ 1, abort_flag, err,
-                                        kDevTimeoutAttn, TO))
-          return false;
+        if (!wait(&bars->p_full[half], Jp & 1)) return false;
         tc_fence_after();
-        const uint32_t t_o = tmem + (ob ? C::TM_O1 : C::TM_O0);
-        const uint32_t t_p = tmem + (sb ? C::TM_S1 : C::TM_S0);
+        const uint32_t t_o = tmem + C::tm_o(half);
+        const uint32_t t_p = tmem + C::tm_s(half);
 #pragma unroll
         for (int ks = 0; ks < kTile / 16; ++ks) {
-          const uint64_t bd =
-              smem_desc_sw128(sVa + st * C::TILE_BYTES + ks * 2048, 16384, 1024);
-          mma_ts(t_o, t_p + ks * 8, bd, IDESC_PV, (first && ks == 0) ? 0u : 1u);
+          const uint64_t bd = smem_desc_sw128(sVa + st * C::HALF_BYTES + ks * 2048, 16384, 1024);
+          mma_ts_elect(t_o, t_p + ks * 8, bd, IDESC_PV, (first && ks == 0) ? 0u : 1u);
         }
-        mma_commit(&bars->v_empty[st]);
-        mma_commit(&bars->o_done);
-        if (last) mma_commit(&bars->o_full[ob]);
+        if (half == 1) mma_commit_elect(&bars->v_empty[st]);
+        if (last) mma_commit_elect(&bars->o_full[half]);
         return true;
       };
+      bool pend = false, pend_first = false, pend_last = false;
+      uint32_t pend_J = 0;
       for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
         const Item it = decode_item(a, w, n_routed);
         if (it.kind == 0) continue;
-        const uint32_t qb = lt & 1;
-        ok = mbar_wait_bounded(&bars->q_full[qb], (lt >> 1) & 1, abort_flag, err, kDevTimeoutAttn, TO);
+        const uint32_t qb = lt % C::QB;
+        if (C::QB == 1 && pend) {  // a single Q buffer: finish the previous item first
+          ok = issue_pv(1, pend_J, pend_first, pend_last);
+          pend = false;
+          if (!ok) break;
+        }
+        ok = wait(&bars->q_full[qb], (lt / C::QB) & 1);
         if (!ok) break;
         tc_fence_after();
         for (int j = 0; j < it.nsub; ++j, ++J) {
-          const uint32_t sb = J & 1;
           const int st = J % C::NST;
-          ok = mbar_wait_bounded(&bars->k_full[st], (J / C::NST) & 1, abort_flag, err, kDevTimeoutAttn, TO);
+          ok = wait(&bars->k_full[st], (J / C::NST) & 1);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t t_s = tmem + (sb ? C::TM_S1 : C::TM_S0);
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-            const uint64_t ad = smem_desc_sw128(sQa + qb * C::TILE_BYTES + off, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(sKa + st * C::TILE_BYTES + off, 16, 1024);
-            mma_ss(t_s, ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
-          }
-          mma_commit(&bars->k_empty[st]);
-          mma_commit(&bars->s_full[sb]);
-          if (j == it.nsub - 1) mma_commit(&bars->q_empty[qb]);
+          issue_s(0, qb, st);
           if (pend) {
-            ok = issue_pv(pend_J, pend_ob, pend_lt, pend_first, pend_last);
+            ok = issue_pv(1, pend_J, pend_first, pend_last);
+            pend = false;
             if (!ok) break;
           }
+          issue_s(1, qb, st);
+          mma_commit_elect(&bars->k_empty[st]);
+          if (j == it.nsub - 1) mma_commit_elect(&bars->q_empty[qb]);
+          ok = wait(&bars->v_full[st], (J / C::NST) & 1);
+          if (!ok) break;
+          ok = issue_pv(0, J, j == 0, j == it.nsub - 1);
+          if (!ok) break;
           pend = true;
           pend_J = J;
-          pend_ob = lt & 1;
-          pend_lt = lt;
           pend_first = (j == 0);
           pend_last = (j == it.nsub - 1);
         }
         ++lt;
       }
-      if (ok && pend) ok = issue_pv(pend_J, pend_ob, pend_lt, pend_first, pend_last);
+      if (ok && pend) ok = issue_pv(1, pend_J, pend_first, pend_last);
       if (!ok) {
         // after an abort, wait (bounded) until the MMAs already issued have finished with TMEM
         volatile int no_abort = 0;
-        mma_commit(&bars->drain);
+        mma_commit_elect(&bars->drain);
         mbar_wait_bounded(&bars->drain, 0, &no_abort, nullptr, 0, TO / 4);
       }
     }
@@ -303,11 +330,11 @@ __global__ void __launch_bounds__(256, 1)
     for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
       const Item it = decode_item(a, w, n_routed);
       if (it.kind == 0) continue;
-      const uint32_t qb = lt & 1;
-      ok = mbar_wait_bounded(&bars->q_empty[qb], ((lt >> 1) & 1) ^ 1, abort_flag, err, kDevTimeoutAttn, TO);
+      const uint32_t qb = lt % C::QB;
+      ok = mbar_wait_bounded(&bars->q_empty[qb], ((lt / C::QB) & 1) ^ 1, abort_flag, err, kDevTimeoutAttn, TO);
       if (!ok) break;
-      const uint32_t dst0 = smem_u32(sQ + qb * C::TILE_BYTES);
-      for (int e = gt; e < kTile * CPR; e += 64) {
+      const uint32_t dst0 = smem_u32(sQ + qb * C::Q_BYTES);
+      for (int e = gt; e < kItemRows * CPR; e += 64) {
         const int m = e / CPR, c = e % CPR;
         const __nv_bfloat16* src = a.q;
         uint32_t bytes = 0;
@@ -324,57 +351,85 @@ __global__ void __launch_bounds__(256, 1)
           src = a.q + (static_cast<size_t>(t) * a.H + h) * D + c * 8;
           bytes = 16;
         }
-        cp_async_16(dst0 + (c >> 3) * 16384 + sw128_offset(m, (c & 7) * 8), src, bytes);
+        const uint32_t dst = dst0 + (m >> 7) * C::HALF_BYTES + (c >> 3) * 16384 +
+                             sw128_offset(m & 127, (c & 7) * 8);
+        cp_async_16(dst, src, bytes);
       }
       cp_async_wait_all();
       fence_proxy_async_smem();
       mbar_arrive(&bars->q_full[qb]);
       ++lt;
     }
+   }
   } else {
+    regs_inc<C::REGS_SOFTMAX>();
     // ------------------------------------------------------------ softmax + epilogue
-    const int row = tid - 128;  // TMEM lane / query row of this thread
-    const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    const int half = (warp >= 8) ? 1 : 0;
+    const int row = tid - 128 - half * 128;  // TMEM lane / row inside the half
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + C::tm_s(half);
+    const uint32_t t_o = tmem + lane_off + C::tm_o(half);
     const float sl2 = a.scale_log2;
     uint32_t J = 0, lt = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
       const Item it = decode_item(a, w, n_routed);
       if (it.kind == 0) continue;
-      const bool valid = row < it.rows;
+      const int r_item = half * kTile + row;  // row inside the 256-row item
+      const bool valid = r_item < it.rows;
       int prow = 0, limit;
       if (it.kind == 1) {
-        if (valid) prow = __ldg(a.entries + it.start + row);
+        if (valid) prow = __ldg(a.entries + it.start + r_item);
         limit = it.klen;
       } else {
-        const int t = it.qtok0 + row;
+        const int t = it.qtok0 + r_item;
         prow = ((t - a.T0) * a.H + it.h) * a.topk + it.slot;
-        limit = valid ? kTile * it.p + row + 1 : 1;
+        limit = valid ? it.qoff + r_item + 1 : 1;
       }
       float m_ref = -INFINITY, l_sum = 0.f;
-      const uint32_t ob = lt & 1;
-      const uint32_t t_o = tmem + lane_off + (ob ? C::TM_O1 : C::TM_O0);
       for (int j = 0; j < it.nsub; ++j, ++J) {
-        const uint32_t sb = J & 1;
-        ok = mbar_wait_bounded(&bars->s_full[sb], (J >> 1) & 1, abort_flag, err, kDevTimeoutAttn, TO);
+        ok = mbar_wait_bounded(&bars->s_full[half], J & 1, abort_flag, err, kDevTimeoutAttn, TO);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t t_s = tmem + lane_off + (sb ? C::TM_S1 : C::TM_S0);
         uint32_t sr[128];
+        const int lim = limit - j * kTile;  // valid columns: c < lim
+        // load S in two halves so the second TMEM load overlaps the first half's max
         tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
         tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 64; ++c) reg_fence(sr[c]);
         tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
         tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-        tmem_wait_ld();
-        const int lim = limit - j * kTile;  // valid columns: c < lim
-        float mx = -INFINITY;
+        if (lim < 64) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float v = (c < lim) ? __uint_as_float(sr[c]) : -INFINITY;
-          sr[c] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
+          for (int c = 0; c < 64; ++c)
+            if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
         }
+        float mx8[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) mx8[x] = __uint_as_float(sr[x]);
+#pragma unroll
+        for (int c = 8; c < 64; c += 8) {
+#pragma unroll
+          for (int x = 0; x < 8; ++x) mx8[x] = fmaxf(mx8[x], __uint_as_float(sr[c + x]));
+        }
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 64; c < 128; ++c) reg_fence(sr[c]);
+        if (lim < kTile) {
+#pragma unroll
+          for (int c = 64; c < 128; ++c)
+            if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
+        }
+#pragma unroll
+        for (int c = 64; c < 128; c += 8) {
+#pragma unroll
+          for (int x = 0; x < 8; ++x) mx8[x] = fmaxf(mx8[x], __uint_as_float(sr[c + x]));
+        }
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float mxs = mx * sl2;
         // raise the reference max only when it grew by more than 2^8 (rare); tcgen05.ld/st are
         // warp-collective, so the O rescale runs for the whole warp (alpha = 1 where not needed)
@@ -386,16 +441,14 @@ __global__ void __launch_bounds__(256, 1)
           m_ref = mxs;
         }
         if (j > 0 && __any_sync(0xffffffffu, need)) {
-          // O holds sub-tiles < j: wait for the PV of sub-tile J-1, then rescale O in TMEM
-          ok = mbar_wait_bounded(&bars->o_done, (J - 1) & 1, abort_flag, err, kDevTimeoutAttn, TO);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          tc_fence_after();
+          // O_x holds sub-tiles < j and is complete (its last PV was issued before this S)
 #pragma unroll
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t orr[32];
             tmem_ld32(t_o + c0, orr);
             tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) reg_fence(orr[x]);
 #pragma unroll
             for (int x = 0; x < 32; ++x) orr[x] = __float_as_uint(__uint_as_float(orr[x]) * alpha);
             tmem_st32(t_o + c0, orr);
@@ -403,25 +456,33 @@ __global__ void __launch_bounds__(256, 1)
           tmem_wait_st();
         }
         const float neg = -m_ref;
-        float ps = 0.f;
-        uint32_t pk[64];
+        float ps8[8];
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, neg));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c + 1]), sl2, neg));
-          ps += p0 + p1;
-          pk[c >> 1] = pack_bf16x2(p0, p1);
+        for (int x = 0; x < 8; ++x) ps8[x] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 128; c += 16) {
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            const float t0 = fmaf(__uint_as_float(sr[c + 2 * x]), sl2, neg);
+            const float t1 = fmaf(__uint_as_float(sr[c + 2 * x + 1]), sl2, neg);
+            // kPolyPairs of every 8 column pairs go to the FMA pipe, the rest to MUFU.EX2
+            const bool poly = x >= 8 - kPolyPairs;
+            const float p0 = poly ? exp2_poly(t0) : ex2_approx(t0);
+            const float p1 = poly ? exp2_poly(t1) : ex2_approx(t1);
+            ps8[x] += p0 + p1;
+            sr[(c >> 1) + x] = pack_bf16x2(p0, p1);  // packed in place: index <= c + 2x
+          }
         }
-        l_sum += ps;
-        tmem_st32(t_s + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(t_s + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+        l_sum += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+        tmem_st32(t_s + 0, *reinterpret_cast<const uint32_t(*)[32]>(&sr[0]));
+        tmem_st32(t_s + 32, *reinterpret_cast<const uint32_t(*)[32]>(&sr[32]));
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->p_full[sb]);
+        mbar_arrive(&bars->p_full[half]);
       }
       if (!ok) break;
       // epilogue: O / l -> bf16 partial row, log-sum-exp
-      ok = mbar_wait_bounded(&bars->o_full[ob], (lt >> 1) & 1, abort_flag, err, kDevTimeoutAttn, TO);
+      ok = mbar_wait_bounded(&bars->o_full[half], lt & 1, abort_flag, err, kDevTimeoutAttn, TO);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -432,6 +493,8 @@ __global__ void __launch_bounds__(256, 1)
         uint32_t orr[32];
         tmem_ld32(t_o + c0, orr);
         tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) reg_fence(orr[x]);
         if (valid) {
           uint4 pkt[4];
           uint32_t* pw = reinterpret_cast<uint32_t*>(pkt);
@@ -444,7 +507,6 @@ __global__ void __launch_bounds__(256, 1)
       }
       if (valid) a.part_lse[prow] = (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
       tc_fence_before();
-      mbar_arrive(&bars->o_free[ob]);
       ++lt;
     }
   }
@@ -512,20 +574,29 @@ cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream) {
   a.b0 = L.b0;
   a.nblk = L.nblk;
   a.T0 = L.T0;
-  a.P = (L.B + kTile - 1) / kTile;
-  a.n_diag = a.P * L.nblk * L.H;
+  a.P2 = (L.B + kItemRows - 1) / kItemRows;
+  a.n_diag = a.P2 * L.nblk * L.H;
   a.scale_log2 = L.scale * 1.4426950408889634f;
   const int grid = L.grid > 0 ? L.grid : 1;
+  // setmaxnreg.inc would wait forever if the launch had fewer registers than the split assumes
+  {
+    cudaFuncAttributes fa;
+    cudaError_t e = (L.d == 64) ? cudaFuncGetAttributes(&fa, attn_kernel<64>)
+                                : cudaFuncGetAttributes(&fa, attn_kernel<128>);
+    if (e != cudaSuccess) return e;
+    const int need = 128 * AttnCfg<128>::REGS_CTRL + 256 * AttnCfg<128>::REGS_SOFTMAX;
+    if (fa.numRegs * 384 < need) return cudaErrorInvalidConfiguration;
+  }
   if (L.d == 64) {
     const int smem = AttnCfg<64>::SMEM_BYTES;
     cudaError_t e = cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_kernel<64><<<grid, 256, smem, stream>>>(mk, mv, a);
+    attn_kernel<64><<<grid, 384, smem, stream>>>(mk, mv, a);
   } else {
     const int smem = AttnCfg<128>::SMEM_BYTES;
     cudaError_t e = cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_kernel<128><<<grid, 256, smem, stream>>>(mk, mv, a);
+    attn_kernel<128><<<grid, 384, smem, stream>>>(mk, mv, a);
   }
   return cudaGetLastError();
 }

@@ -6,7 +6,8 @@
 
 namespace moba {
 
-constexpr int kTile = 128;           // query rows per attention tile, keys per key sub-tile
+constexpr int kTile = 128;           // rows of one MMA half-tile, keys per key sub-tile
+constexpr int kItemRows = 256;       // query rows per attention work item (two 128-row halves)
 constexpr int kMaxTopk = 64;
 constexpr int kMaxBlocksPerSeq = 32768;
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s per bounded device wait

@@ -5,8 +5,8 @@
 // gathered from scattered rows into one dense operand [FlashMoBA story, Gather-and-Densify]. The
 // inversion is a counting sort of the routed (t, h, slot) triples by bucket (g, b):
 //   route_count   : per-CTA shared-memory histograms, one global atomic per (CTA, bucket);
-//   route_scan    : exclusive scan of the bucket counts -> list offsets, and the list of 128-row
-//                   attention tiles (bucket, first entry, rows);
+//   route_scan    : exclusive scan of the bucket counts -> list offsets, and the list of 256-row
+//                   attention work items (bucket, first entry, rows);
 //   route_scatter : per-CTA reservation of a contiguous range per bucket, then shared-memory
 //                   cursors place every entry.
 // An entry is the index of the partial-output row of (t, h, slot): ((t - T0) * Hq + h) * k + slot,
@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(256) route_pass_kernel(
   }
 }
 
-// One CTA of 1024 threads: offsets, cursors and the 128-row tile list of every bucket; resets the
+// One CTA of 1024 threads: offsets, cursors and the 256-row work-item list of every bucket; resets the
 // bucket counters for the next chunk.
 __global__ void __launch_bounds__(1024) route_scan_kernel(int* __restrict__ counts, int nbk,
                                                           int* __restrict__ cursor,
@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int* __restrict__ coun
   for (int x = k0; x < k1; ++x) {
     const int c = counts[x];
     lc += c;
-    lt += (c + kTile - 1) / kTile;
+    lt += (c + kItemRows - 1) / kItemRows;
   }
   int ic = lc, it = lt;
 #pragma unroll
@@ -182,9 +182,9 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int* __restrict__ coun
   for (int x = k0; x < k1; ++x) {
     const int c = counts[x];
     cursor[x] = off;
-    for (int y = 0; y * kTile < c; ++y)
-      tiles[toff + y] = make_int4(x, off + y * kTile, min(kTile, c - y * kTile), 0);
-    toff += (c + kTile - 1) / kTile;
+    for (int y = 0; y * kItemRows < c; ++y)
+      tiles[toff + y] = make_int4(x, off + y * kItemRows, min(kItemRows, c - y * kItemRows), 0);
+    toff += (c + kItemRows - 1) / kItemRows;
     off += c;
     counts[x] = 0;
   }

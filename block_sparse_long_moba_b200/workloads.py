@@ -66,6 +66,9 @@ WORKLOADS = {
     "routing_64k_b128": Workload("routing_64k_b128", [0, 65536], 16, 16, 64, 128, 16, "clusters"),
     "varlen_512k_b128": Workload("varlen_512k_b128", [0, 65536, 196608, 294912, 524288],
                                  16, 16, 64, 128, 32, "clusters"),
+    # small cases of the same kernels for profiler captures (a few GB on the device)
+    "profile_32k_b4096": Workload("profile_32k_b4096", [0, 32768], 32, 8, 128, 4096, 4, "offset"),
+    "profile_32k_b128": Workload("profile_32k_b128", [0, 32768], 16, 16, 64, 128, 16, "clusters"),
 }
 WORKLOAD_ORDER = ["tiny_1k", "llama8b_128k", "llama8b_1m", "routing_64k_b128", "varlen_512k_b128"]
 
