@@ -35,6 +35,10 @@ namespace moba {
 
 // Column pairs (of every 8) whose exp2 runs on the FMA pipe instead of MUFU.EX2, balancing the two.
 constexpr int kPolyPairs = 0;
+#ifndef MOBA_POLY_PAIRS_PVT
+#define MOBA_POLY_PAIRS_PVT 0
+#endif
+constexpr int kPolyPairsPvt = MOBA_POLY_PAIRS_PVT;
 
 struct AttnArgs {
   const __nv_bfloat16* q;  // [T, H, D]
@@ -519,6 +523,451 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// d = 128: P staged in shared memory, PV computed transposed for both halves at once.
+//
+// On B200 a 128 x N x 16 tcgen05.mma issued back to back costs ~100 cycles for any N <= 128
+// (measured) but reaches the nominal 128 cycles at N = 256. Here the two 128-row halves A and B
+// keep their own S = Q K^T (M = 128, N = 128 keys), but P = exp(...) goes to shared memory and
+// the value product is computed as O^T = V^T P^T: M = d = 128, N = 256 queries (both halves),
+// K = 128 keys — eight full-rate instructions per sub-tile instead of sixteen half-rate ones.
+// Since P no longer aliases S in tensor memory, S_x(j+1) is issued as soon as the softmax has
+// read S_x(j), so QK^T of the next sub-tile overlaps this sub-tile's softmax.
+// Tensor memory: S_A [0,128), S_B [128,256), O^T [256,512) (lanes = d, columns = the 256 rows).
+// O^T columns are rescaled (rarely) by the warpgroup that owns those rows, between PV(j-1) and
+// PV(j); the epilogue normalises O^T by l, transposes it through shared memory and writes rows.
+struct PvtCfg {
+  static constexpr int D = 128;
+  static constexpr int HALF_BYTES = kTile * D * 2;  // 32 KB
+  static constexpr int Q_BYTES = 2 * HALF_BYTES;     // 64 KB (one buffer)
+  static constexpr int NSTK = 2;                     // K ring
+  static constexpr int P_BYTES = 2 * HALF_BYTES;     // 256 rows x 128 keys bf16
+  static constexpr int OFF_K = Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NSTK * HALF_BYTES;
+  static constexpr int OFF_P = OFF_V + HALF_BYTES;   // single V stage
+  static constexpr int OFF_ALPHA = OFF_P + P_BYTES;  // float[256]
+  static constexpr int OFF_INVL = OFF_ALPHA + 1024;  // float[256]
+  static constexpr int OFF_BARS = OFF_INVL + 1024;
+  static constexpr int SMEM_BYTES = OFF_BARS + 256;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t TM_OT = 256;
+  static constexpr uint32_t REGS_CTRL = 72, REGS_SOFTMAX = 216;
+  __host__ __device__ static constexpr uint32_t tm_s(int x) { return 128u * x; }
+};
+static_assert(PvtCfg::SMEM_BYTES <= 232448, "shared memory budget of one CTA");
+
+struct PvtBars {
+  uint64_t q_full, q_empty;
+  uint64_t k_full[2], k_empty[2], v_full, v_empty;
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full, pv_done;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(PvtBars) <= 256, "barrier block");
+
+// Walks the 128-key sub-tiles of this CTA's work items in order (empty items skipped).
+struct SubTileCursor {
+  int w = -1, j = 0;
+  Item it;
+  __device__ __forceinline__ bool next(const AttnArgs& a, int n_items, int n_routed) {
+    if (w >= 0 && ++j < it.nsub) return true;
+    for (w = (w < 0) ? static_cast<int>(blockIdx.x) : w + static_cast<int>(gridDim.x); w < n_items;
+         w += gridDim.x) {
+      it = decode_item(a, w, n_routed);
+      if (it.kind != 0) {
+        j = 0;
+        return true;
+      }
+    }
+    return false;
+  }
+};
+
+// Byte offset of element (row, col) in a 256-row operand stored as two 64-column blocks of
+// 256 x 128 bytes with the 128-byte swizzle (the P layout, also used to stage O rows).
+__device__ __forceinline__ uint32_t p_offset(uint32_t row, uint32_t col) {
+  return (col >> 6) * 32768u + sw128_offset(row, col & 63u);
+}
+
+__global__ void __launch_bounds__(384, 1)
+    attn_kernel_pvt(const __grid_constant__ CUtensorMap map_k,
+                    const __grid_constant__ CUtensorMap map_v, const AttnArgs a) {
+  using C = PvtCfg;
+  constexpr int D = C::D;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  uint8_t* sP = smem + C::OFF_P;
+  float* s_alpha = reinterpret_cast<float*>(smem + C::OFF_ALPHA);
+  float* s_invl = reinterpret_cast<float*>(smem + C::OFF_INVL);
+  PvtBars* bars = reinterpret_cast<PvtBars*>(smem + C::OFF_BARS);
+  volatile int* abort_flag = &bars->abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the swizzled layouts assume a 1024-byte aligned base: refuse to run otherwise
+  if (smem_u32(smem) & 1023u) {
+    if (tid == 0) atomicCAS(a.status, 0, kDevTimeoutAttn);
+    return;
+  }
+  if (tid == 0) {
+    mbar_init(&bars->q_full, 64);
+    mbar_init(&bars->q_empty, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->k_full[x], 1);
+      mbar_init(&bars->k_empty[x], 1);
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->s_free[x], 128);
+    }
+    mbar_init(&bars->v_full, 1);
+    mbar_init(&bars->v_empty, 1);
+    mbar_init(&bars->p_full, 256);
+    mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&map_k);
+    prefetch_tensormap(&map_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const int n_routed = *a.n_routed;
+  const int n_items = n_routed + a.n_diag;
+  const uint64_t TO = kWaitTimeoutNs;
+  int* err = a.status;
+
+  if (warp < 4) {
+    regs_dec<C::REGS_CTRL>();
+    if (warp == 0) {
+      // -------------------------------------------------------------- TMA producer (K, V)
+      // K runs up to two sub-tiles ahead of V: the next QK^T is issued before this PV, and the
+      // single V stage only frees up when the previous PV has completed.
+      SubTileCursor ck, cv;
+      bool hk = ck.next(a, n_items, n_routed), hv = cv.next(a, n_items, n_routed);
+      uint32_t JK = 0, JV = 0;
+      bool ok = true;
+      while (ok && (hk || hv)) {
+        if (hk && (JK < JV + 2 || !hv)) {
+          const int st = JK & 1;
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->k_empty[st], ((JK >> 1) & 1) ^ 1,
+                                                         abort_flag, err, kDevTimeoutAttn, TO));
+          if (!ok) break;
+          const int tok = ck.it.key0 + ck.j * kTile;
+          mbar_arrive_expect_tx_elect(&bars->k_full[st], C::HALF_BYTES);
+          tma_load_3d_elect(sK + st * C::HALF_BYTES, &map_k, &bars->k_full[st], 0, ck.it.g, tok);
+          tma_load_3d_elect(sK + st * C::HALF_BYTES + 16384, &map_k, &bars->k_full[st], 64,
+                            ck.it.g, tok);
+          ++JK;
+          hk = ck.next(a, n_items, n_routed);
+        } else {
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->v_empty, (JV & 1) ^ 1, abort_flag,
+                                                         err, kDevTimeoutAttn, TO));
+          if (!ok) break;
+          const int tok = cv.it.key0 + cv.j * kTile;
+          mbar_arrive_expect_tx_elect(&bars->v_full, C::HALF_BYTES);
+          tma_load_3d_elect(sV, &map_v, &bars->v_full, 0, cv.it.g, tok);
+          tma_load_3d_elect(sV + 16384, &map_v, &bars->v_full, 64, cv.it.g, tok);
+          ++JV;
+          hv = cv.next(a, n_items, n_routed);
+        }
+      }
+      if (!ok) {
+        volatile int no_abort = 0;
+        for (uint32_t x = 0; x < 2; ++x) {
+          if (JK > x) {
+            const uint32_t Jx = JK - 1 - x;
+            mbar_wait_bounded(&bars->k_full[Jx & 1], (Jx >> 1) & 1, &no_abort, nullptr, 0, TO / 4);
+          }
+        }
+        if (JV > 0) mbar_wait_bounded(&bars->v_full, (JV - 1) & 1, &no_abort, nullptr, 0, TO / 4);
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t IDESC_PVT = idesc_bf16_f32(128, 256, 1, 0);  // A = V^T (MN-major)
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV), sPa = smem_u32(sP);
+      bool ok = true;
+      auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu,
+                          mbar_wait_bounded(bar, parity, abort_flag, err, kDevTimeoutAttn, TO));
+      };
+      // S_x(J) = Q_x K_J^T; the S_x buffer must have been read by the softmax of sub-tile J-1
+      auto issue_s = [&](int x, uint32_t J) -> bool {
+        if (J > 0 && !wait(&bars->s_free[x], (J - 1) & 1)) return false;
+        tc_fence_after();
+        const int st = J & 1;
+        const uint32_t qbase = sQa + x * C::HALF_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_ss_elect(tmem + C::tm_s(x), smem_desc_sw128(qbase + off, 16, 1024),
+                       smem_desc_sw128(sKa + st * C::HALF_BYTES + off, 16, 1024), IDESC_QK,
+                       ks > 0 ? 1u : 0u);
+        }
+        mma_commit_elect(&bars->s_full[x]);
+        return true;
+      };
+      auto issue_s_pair = [&](uint32_t J, bool last_of_item) -> bool {
+        if (!wait(&bars->k_full[J & 1], (J >> 1) & 1)) return false;
+        tc_fence_after();
+        if (!issue_s(0, J) || !issue_s(1, J)) return false;
+        mma_commit_elect(&bars->k_empty[J & 1]);
+        if (last_of_item) mma_commit_elect(&bars->q_empty);
+        return true;
+      };
+      // O^T (+)= V_J^T P_J^T for both halves
+      auto issue_pvt = [&](uint32_t J, bool first) -> bool {
+        if (!wait(&bars->v_full, J & 1)) return false;
+        if (!wait(&bars->p_full, J & 1)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < kTile / 16; ++ks) {
+          const uint64_t ad = smem_desc_sw128(sVa + ks * 2048, 16384, 1024);
+          const uint64_t bd = smem_desc_sw128(sPa + (ks >> 2) * 32768 + (ks & 3) * 32, 16, 1024);
+          mma_ss_elect(tmem + C::TM_OT, ad, bd, IDESC_PVT, (first && ks == 0) ? 0u : 1u);
+        }
+        mma_commit_elect(&bars->v_empty);
+        mma_commit_elect(&bars->pv_done);
+        return true;
+      };
+      uint32_t J = 0, lt = 0;
+      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+        const Item it = decode_item(a, w, n_routed);
+        if (it.kind == 0) continue;
+        ok = wait(&bars->q_full, lt & 1);
+        if (!ok) break;
+        tc_fence_after();
+        ok = issue_s_pair(J, it.nsub == 1);
+        for (int j = 0; j < it.nsub && ok; ++j) {
+          if (j + 1 < it.nsub) {
+            ok = issue_s_pair(J + j + 1, j + 1 == it.nsub - 1);
+            if (!ok) break;
+          }
+          ok = issue_pvt(J + j, j == 0);
+        }
+        J += it.nsub;
+        ++lt;
+      }
+      if (!ok) {
+        volatile int no_abort = 0;
+        mma_commit_elect(&bars->drain);
+        mbar_wait_bounded(&bars->drain, 0, &no_abort, nullptr, 0, TO / 4);
+      }
+    } else {
+      // ------------------------------------------------------------------ Q row gather
+      const int gt = tid - 64;  // 0..63
+      constexpr int CPR = D / 8;
+      uint32_t lt = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+        const Item it = decode_item(a, w, n_routed);
+        if (it.kind == 0) continue;
+        ok = mbar_wait_bounded(&bars->q_empty, (lt & 1) ^ 1, abort_flag, err, kDevTimeoutAttn, TO);
+        if (!ok) break;
+        const uint32_t dst0 = smem_u32(sQ);
+        for (int e = gt; e < kItemRows * CPR; e += 64) {
+          const int m = e / CPR, c = e % CPR;
+          const __nv_bfloat16* src = a.q;
+          uint32_t bytes = 0;
+          if (m < it.rows) {
+            int t, h;
+            if (it.kind == 1) {
+              const int pr = __ldg(a.entries + it.start + m);
+              t = a.T0 + pr / (a.H * a.topk);
+              h = (pr / a.topk) % a.H;
+            } else {
+              t = it.qtok0 + m;
+              h = it.h;
+            }
+            src = a.q + (static_cast<size_t>(t) * a.H + h) * D + c * 8;
+            bytes = 16;
+          }
+          const uint32_t dst = dst0 + (m >> 7) * C::HALF_BYTES + (c >> 3) * 16384 +
+                               sw128_offset(m & 127, (c & 7) * 8);
+          cp_async_16(dst, src, bytes);
+        }
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->q_full);
+        ++lt;
+      }
+    }
+  } else {
+    regs_inc<C::REGS_SOFTMAX>();
+    // -------------------------------------------------------------- softmax + epilogue
+    const int half = (warp >= 8) ? 1 : 0;
+    const int row = tid - 128 - half * 128;          // TMEM lane; row of this half
+    const int q = half * kTile + row;                 // row of the 256-row item
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + C::tm_s(half);
+    const uint32_t t_ot = tmem + lane_off + C::TM_OT + half * kTile;  // this half's O^T columns
+    const uint32_t bar_id = 1 + half;                 // named barrier of this warpgroup
+    const float sl2 = a.scale_log2;
+    uint32_t J = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+      const Item it = decode_item(a, w, n_routed);
+      if (it.kind == 0) continue;
+      const bool valid = q < it.rows;
+      int prow = 0, limit;
+      if (it.kind == 1) {
+        if (valid) prow = __ldg(a.entries + it.start + q);
+        limit = it.klen;
+      } else {
+        const int t = it.qtok0 + q;
+        prow = ((t - a.T0) * a.H + it.h) * a.topk + it.slot;
+        limit = valid ? it.qoff + q + 1 : 1;
+      }
+      float m_ref = -INFINITY, l_sum = 0.f;
+      for (int j = 0; j < it.nsub; ++j, ++J) {
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[half], J & 1, abort_flag,
+                                                       err, kDevTimeoutAttn, TO));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sr[128];
+        const int lim = limit - j * kTile;
+        tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+        tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 128; ++c) reg_fence(sr[c]);
+        tc_fence_before();
+        mbar_arrive(&bars->s_free[half]);  // S_x may now be overwritten by the next QK^T
+        if (lim < kTile) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
+        }
+        float mx8[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) mx8[x] = __uint_as_float(sr[x]);
+#pragma unroll
+        for (int c = 8; c < 128; c += 8) {
+#pragma unroll
+          for (int x = 0; x < 8; ++x) mx8[x] = fmaxf(mx8[x], __uint_as_float(sr[c + x]));
+        }
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float mxs = mx * sl2;
+        const bool need = mxs > m_ref + 8.f;
+        float alpha = 1.f;
+        if (need) {
+          alpha = ex2_approx(m_ref - mxs);
+          l_sum *= alpha;
+          m_ref = mxs;
+        }
+        const float neg = -m_ref;
+        // p = exp2(s * scale * log2e - m) for a column pair, packed to bf16x2; pair sums in f32x2
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+        auto exp_pair = [&](int c) -> uint32_t {
+          float t0, t1;
+          fma2(t0, t1, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), sl2, sl2, neg, neg);
+          const bool poly = ((c >> 1) & 7) >= 8 - kPolyPairsPvt;
+          const float p0 = poly ? exp2_poly(t0) : ex2_approx(t0);
+          const float p1 = poly ? exp2_poly(t1) : ex2_approx(t1);
+          const int x = (c >> 1) & 3;
+          add2(sa[x], sb[x], sa[x], sb[x], p0, p1);
+          return pack_bf16x2(p0, p1);
+        };
+        // columns 0..63 first, held packed in sr[0..31]
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) sr[c >> 1] = exp_pair(c);
+        // P(J) reuses the shared P tile: PV(J-1) must be complete (it also fixes O^T for a rescale)
+        if (J > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done, (J - 1) & 1, abort_flag,
+                                                         err, kDevTimeoutAttn, TO));
+          if (!ok) break;
+        }
+        s_alpha[q] = alpha;
+        if (named_bar_or(bar_id, 128, need && j > 0)) {
+          // some row of this half raised its max: scale this half's O^T columns (lane = d)
+          tc_fence_after();
+#pragma unroll 1
+          for (int c0 = 0; c0 < kTile; c0 += 32) {
+            uint32_t orr[32];
+            tmem_ld32(t_ot + c0, orr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) reg_fence(orr[x]);
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+              orr[x] = __float_as_uint(__uint_as_float(orr[x]) * s_alpha[half * kTile + c0 + x]);
+            tmem_st32(t_ot + c0, orr);
+          }
+          tmem_wait_st();
+        }
+        // P row q -> shared memory (K-major, 128-byte swizzle); the second half of the row is
+        // computed and stored chunk by chunk so the stores overlap the exponentials
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(sP + p_offset(q, c * 8)) =
+              make_uint4(sr[4 * c], sr[4 * c + 1], sr[4 * c + 2], sr[4 * c + 3]);
+#pragma unroll
+        for (int c = 64; c < 128; c += 8) {
+          const uint32_t w0 = exp_pair(c), w1 = exp_pair(c + 2), w2 = exp_pair(c + 4),
+                         w3 = exp_pair(c + 6);
+          *reinterpret_cast<uint4*>(sP + p_offset(q, c)) = make_uint4(w0, w1, w2, w3);
+        }
+        l_sum += ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full);
+      }
+      if (!ok) break;
+      // ---- epilogue: O = O^T / l, transposed through the (now idle) P tile
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done, (J - 1) & 1, abort_flag, err,
+                                                     kDevTimeoutAttn, TO));
+      if (!ok) break;
+      tc_fence_after();
+      s_invl[q] = (valid && l_sum > 0.f) ? 1.f / l_sum : 0.f;
+      named_bar_sync(bar_id, 128);
+      // thread `row` holds O^T lane d = row: columns are this half's 128 query rows
+#pragma unroll 1
+      for (int c0 = 0; c0 < kTile; c0 += 32) {
+        uint32_t orr[32];
+        tmem_ld32(t_ot + c0, orr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) reg_fence(orr[x]);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const int qq = half * kTile + c0 + x;
+          const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(orr[x]) * s_invl[qq]);
+          *reinterpret_cast<__nv_bfloat16*>(sP + p_offset(qq, row)) = b;
+        }
+      }
+      named_bar_sync(bar_id, 128);
+      if (valid) {
+        __nv_bfloat16* dst = a.part_o + static_cast<size_t>(prow) * D;
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          reinterpret_cast<uint4*>(dst)[c] = *reinterpret_cast<const uint4*>(sP + p_offset(q, c * 8));
+        a.part_lse[prow] = (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
+      }
+      // the P tile rows of this half are rewritten only by this warpgroup, after this point
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
 // ---------------------------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -582,7 +1031,7 @@ cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream) {
   {
     cudaFuncAttributes fa;
     cudaError_t e = (L.d == 64) ? cudaFuncGetAttributes(&fa, attn_kernel<64>)
-                                : cudaFuncGetAttributes(&fa, attn_kernel<128>);
+                                : cudaFuncGetAttributes(&fa, attn_kernel_pvt);
     if (e != cudaSuccess) return e;
     const int need = 128 * AttnCfg<128>::REGS_CTRL + 256 * AttnCfg<128>::REGS_SOFTMAX;
     if (fa.numRegs * 384 < need) return cudaErrorInvalidConfiguration;
@@ -593,10 +1042,10 @@ cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attn_kernel<64><<<grid, 384, smem, stream>>>(mk, mv, a);
   } else {
-    const int smem = AttnCfg<128>::SMEM_BYTES;
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int smem = PvtCfg::SMEM_BYTES;
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel_pvt, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_kernel<128><<<grid, 384, smem, stream>>>(mk, mv, a);
+    attn_kernel_pvt<<<grid, 384, smem, stream>>>(mk, mv, a);
   }
   return cudaGetLastError();
 }
