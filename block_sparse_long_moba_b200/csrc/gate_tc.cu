@@ -1,0 +1,412 @@
+// K2 on the tensor cores — parameter-less causal top-k gate [MoBA paper summary (atlas.scime.ai),
+// "Approach"; MoBA README, "Parameter-less Gating Mechanism"].
+//
+// Scores of one tile of 128 query rows (128 consecutive tokens of one query head) against the past
+// blocks of their sequence are one matrix product on tcgen05:
+//   S[128, n] = Q[128, d] . C[n, d]^T,  C = c_hi + c_lo  (two bf16 terms of the fp32 centroids)
+// so each fp32 centroid enters with ~2^-17 relative error and every product q * c_part is exact
+// in the fp32 accumulator. The T x NB score matrix never exists in memory [FlashMoBA story,
+// FlashTopK]: up to 256 scores per row at a time live in tensor memory.
+//
+// Selection: one thread per row (= TMEM lane) keeps its running top list in registers, sorted
+// best first (strict comparison, so equal scores keep the lower block). Scores are read 32 at a
+// time, staged in shared memory, and each row visits only the columns that beat its current
+// threshold, so a warp pays for the largest per-row candidate count of a chunk rather than for
+// every column.
+//
+// A CTA holds two warpgroups (one query tile each) and works on one (query block, kv head) unit at a
+// time: the split centroids of the unit's past blocks are converted into shared memory once and
+// reused by all r * B / 128 tiles of the unit when they fit, and streamed in chunks otherwise.
+#include "common.cuh"
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace moba {
+
+namespace {
+
+constexpr int kTilesPerUnit = 16;  // query tiles that share one conversion of the centroids
+
+template <int D>
+struct GateCfg {
+  static constexpr int NCB = D / 64;
+  static constexpr int Q_BYTES = kTile * D * 2;             // one 128-row query tile
+  static constexpr int CAP = (D == 128) ? 256 : 640;         // centroid rows resident at once
+  static constexpr int B_BYTES = 2 * NCB * CAP * 128;        // hi + lo, 128 B per row per block
+  static constexpr int OFF_B = 2 * Q_BYTES;                  // one Q buffer per warpgroup
+  static constexpr int OFF_STAGE = OFF_B + B_BYTES;          // [2][32][128] staged scores
+  static constexpr int OFF_BARS = OFF_STAGE + 2 * 32 * 128 * 4;
+  static constexpr int SMEM_BYTES = OFF_BARS + 256;
+  static constexpr int PIECE = 256;                          // MMA N (scores per TMEM pass)
+};
+static_assert(GateCfg<128>::SMEM_BYTES <= 232448 && GateCfg<64>::SMEM_BYTES <= 232448,
+              "shared memory budget of one CTA");
+
+struct GateBars {
+  uint64_t q_full[2], mma_done[2];
+  uint32_t tmem_base;
+  int abort_flag;
+  int red[32];
+};
+
+template <int D>
+__device__ __forceinline__ uint32_t c_offset(int s, int row, int col) {
+  using C = GateCfg<D>;
+  return static_cast<uint32_t>(s * C::NCB * C::CAP * 128 + (col >> 6) * C::CAP * 128) +
+         sw128_offset(row, col & 63);
+}
+
+template <int KCAP>
+__device__ __forceinline__ void insert_top(float (&vals)[KCAP], int (&ids)[KCAP], float s, int j) {
+  vals[KCAP - 1] = s;
+  ids[KCAP - 1] = j;
+#pragma unroll
+  for (int x = KCAP - 1; x > 0; --x) {
+    if (vals[x] > vals[x - 1]) {
+      const float tv = vals[x];
+      vals[x] = vals[x - 1];
+      vals[x - 1] = tv;
+      const int ti = ids[x];
+      ids[x] = ids[x - 1];
+      ids[x - 1] = ti;
+    }
+  }
+}
+
+}  // namespace
+
+template <int D, int KCAP>
+__global__ void __launch_bounds__(256, 1)
+    gate_tc_kernel(const __grid_constant__ CUtensorMap map_q, const float* __restrict__ cents,
+                   const int32_t* __restrict__ cu, int nseq, int max_nb, int T, int H, int G,
+                   int B, int topk, int32_t* __restrict__ idx, int* __restrict__ status) {
+  using C = GateCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  GateBars* bars = reinterpret_cast<GateBars*>(smem + C::OFF_BARS);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int wg = tid >> 7, row = tid & 127;
+  if (smem_u32(smem) & 1023u) {  // swizzled layouts need a 1024-byte aligned base
+    if (tid == 0 && status) atomicCAS(status, 0, kDevTimeoutAttn);
+    return;
+  }
+  volatile int* abort_flag = &bars->abort_flag;
+  if (tid == 0) {
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->q_full[x], 1);
+      mbar_init(&bars->mma_done[x], 1);
+    }
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) prefetch_tensormap(&map_q);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const uint32_t t_s = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + wg * C::PIECE;
+  uint8_t* sQ = smem + wg * C::Q_BYTES;
+  float* stage = reinterpret_cast<float*>(smem + C::OFF_STAGE) + wg * 32 * 128;  // [x][row]
+  const uint32_t sBa = smem_u32(smem + C::OFF_B);
+  const int r = H / G;
+  const int ksel = topk - 1;
+  const uint64_t TO = kWaitTimeoutNs;
+  uint32_t qphase = 0, mphase = 0;  // barrier phases of this warpgroup
+  bool ok = true;
+
+  // Work units: (sequence, kv head g, group of QG consecutive query blocks, sub-range of at most
+  // kTilesPerUnit tiles). Tiles of a unit share the centroid prefix [0, i_max) of its last query
+  // block; each tile only considers its own past blocks j < i. Every wait is bounded; `ok` is made
+  // uniform at each barrier (CTA-wide __syncthreads_and, warpgroup-wide bar.red.and) so that a
+  // timeout never leaves a barrier half-attended.
+  const int ttiles_max = (B + kTile - 1) / kTile;
+  const int tiles_per_block = r * ttiles_max;
+  const int QG = max(1, kTilesPerUnit / tiles_per_block);      // query blocks per unit
+  const int n_sub = (QG * tiles_per_block + kTilesPerUnit - 1) / kTilesPerUnit;
+  const int n_groups = (max_nb + QG - 1) / QG;
+  const long long n_units = static_cast<long long>(nseq) * G * n_groups * n_sub;
+  for (long long u = blockIdx.x; u < n_units; u += gridDim.x) {
+    const int sub = static_cast<int>(u % n_sub);
+    long long rest = u / n_sub;
+    const int ig = static_cast<int>(rest % n_groups);
+    rest /= n_groups;
+    const int g = static_cast<int>(rest % G);
+    const int s = static_cast<int>(rest / G);
+    const int seq0 = cu[s], L = cu[s + 1] - seq0;
+    const int nb = blocks_of(L, B);
+    const int i_first = ig * QG;
+    if (i_first >= nb) continue;  // uniform over the CTA
+    const int i_last = min(nb, i_first + QG) - 1;
+    // tiles of the unit: query blocks i_first..i_last, r heads, 128-token tiles of each block
+    const int nt_all = (i_last - i_first + 1) * tiles_per_block;
+    const int tile_lo = sub * kTilesPerUnit;
+    if (tile_lo >= nt_all) continue;
+    const int ntiles = min(kTilesPerUnit, nt_all - tile_lo);
+    auto tile_info = [&](int tile, int& i_t, int& h_t, int& t0_t, int& rows_t) {
+      const int tg = tile_lo + tile;
+      const int ib = tg / tiles_per_block, w = tg % tiles_per_block;
+      i_t = i_first + ib;
+      h_t = g * r + w / ttiles_max;
+      const int tt = w % ttiles_max;
+      const int blen = min(B, L - i_t * B);
+      t0_t = seq0 + i_t * B + tt * kTile;
+      rows_t = max(0, min(kTile, blen - tt * kTile));
+    };
+    // past blocks needed by the unit: [0, i_max) with i_max the largest scored query block
+    const int i_max = i_last > ksel && ksel > 0 ? i_last : 0;
+    const int base = seq_block_base(cu, s, B, bars->red);
+    const int nchunks = (i_max + C::CAP - 1) / C::CAP;
+    auto load_q = [&](int tile) {  // TMA of a query tile into this warpgroup's buffer
+      int i_t, h_t, t0_t, rows_t;
+      tile_info(tile, i_t, h_t, t0_t, rows_t);
+      mbar_arrive_expect_tx(&bars->q_full[wg], C::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < C::NCB; ++c)
+        tma_load_3d(sQ + c * 16384, &map_q, &bars->q_full[wg], c * 64, h_t, t0_t);
+    };
+    // the first tile of each warpgroup that needs scores
+    auto next_scored = [&](int from) {
+      for (int t = from; t < ntiles; t += 2) {
+        int i_t, h_t, t0_t, rows_t;
+        tile_info(t, i_t, h_t, t0_t, rows_t);
+        if (rows_t > 0 && i_t > ksel && ksel > 0) return t;
+      }
+      return ntiles;
+    };
+    if (row == 0 && ok) {
+      const int t = next_scored(wg);
+      if (t < ntiles) load_q(t);
+    }
+    // tiles are processed in pairs (one per warpgroup); every chunk of centroids is shared
+    for (int p = 0; p < (ntiles + 1) / 2; ++p) {
+      const int tile = 2 * p + wg;
+      int i_t = 0, h = 0, t0 = 0, rows = 0;
+      if (tile < ntiles) tile_info(tile, i_t, h, t0, rows);
+      const bool scored = tile < ntiles && rows > 0 && i_t > ksel && ksel > 0;
+      if (tile < ntiles && rows > 0 && !scored && row < rows) {
+        // few causal blocks or topk == 1: the selection is fixed, no scores needed
+        int32_t* out = idx + (static_cast<size_t>(h) * T + t0 + row) * topk;
+        if (ksel == 0) out[0] = i_t;
+        else
+          for (int x = 0; x < topk; ++x) out[x] = (x <= i_t) ? x : -1;
+      }
+      float vals[KCAP];
+      int ids[KCAP];
+#pragma unroll
+      for (int x = 0; x < KCAP; ++x) {
+        vals[x] = -INFINITY;
+        ids[x] = 0x7fffffff;
+      }
+      bool q_ready = false;
+      for (int ch = 0; ch < nchunks; ++ch) {
+        const int c0 = ch * C::CAP;
+        const int n = min(C::CAP, i_max - c0);
+        if (nchunks > 1 || p == 0) {
+          // split the fp32 centroids of blocks [c0, c0 + n) into hi / lo bf16 tiles
+          ok = __syncthreads_and(ok);
+          const int nrows = (n + 15) & ~15;
+          for (int e = tid; ok && e < nrows * (D / 8); e += blockDim.x) {
+            const int rr = e / (D / 8), c8 = (e % (D / 8)) * 8;
+            uint4 hi = make_uint4(0, 0, 0, 0), lo = make_uint4(0, 0, 0, 0);
+            if (rr < n) {
+              const float4* src = reinterpret_cast<const float4*>(
+                  cents + (static_cast<size_t>(base + c0 + rr) * G + g) * D + c8);
+              const float4 a0 = __ldg(src), a1 = __ldg(src + 1);
+              const float x[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+              uint32_t hw[4], lw[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * k]);
+                const __nv_bfloat16 h1 = __float2bfloat16_rn(x[2 * k + 1]);
+                const __nv_bfloat16 l0 = __float2bfloat16_rn(x[2 * k] - __bfloat162float(h0));
+                const __nv_bfloat16 l1 = __float2bfloat16_rn(x[2 * k + 1] - __bfloat162float(h1));
+                hw[k] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                        (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+                lw[k] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
+                        (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+              }
+              hi = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              lo = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+            *reinterpret_cast<uint4*>(smem + C::OFF_B + c_offset<D>(0, rr, c8)) = hi;
+            *reinterpret_cast<uint4*>(smem + C::OFF_B + c_offset<D>(1, rr, c8)) = lo;
+          }
+          fence_proxy_async_smem();
+          __syncthreads();
+        }
+        if (!scored || c0 >= i_t) continue;  // warpgroup-uniform
+        const int n_t = min(n, i_t - c0);       // this tile's past blocks in the chunk
+        if (!q_ready) {
+          const bool w = ok && mbar_wait_bounded(&bars->q_full[wg], qphase, abort_flag, status,
+                                                 kDevTimeoutAttn, TO);
+          qphase ^= 1;
+          q_ready = true;
+          ok = named_bar_and(1 + wg, 128, w);
+        }
+        // scores of this chunk in passes of up to 256 blocks
+        for (int p0 = 0; p0 < n_t; p0 += C::PIECE) {
+          const int np = min(C::PIECE, n_t - p0);
+          const int nmma = (np + 15) & ~15;
+          if (ok && warp == wg * 4) {  // one converged warp of the warpgroup issues
+            tc_fence_after();
+            const uint32_t idesc = idesc_bf16_f32(128, nmma, 0, 0);
+            const uint32_t qa = smem_u32(sQ);
+#pragma unroll
+            for (int sp = 0; sp < 2; ++sp) {
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t aoff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                const uint32_t boff = static_cast<uint32_t>(sp * C::NCB * C::CAP * 128 +
+                                                            (ks >> 2) * C::CAP * 128 + p0 * 128 +
+                                                            (ks & 3) * 32);
+                mma_ss_elect(tmem + wg * C::PIECE, smem_desc_sw128(qa + aoff, 16, 1024),
+                             smem_desc_sw128(sBa + boff, 16, 1024), idesc,
+                             (sp > 0 || ks > 0) ? 1u : 0u);
+              }
+            }
+            mma_commit_elect(&bars->mma_done[wg]);
+          }
+          const bool w = ok && mbar_wait_bounded(&bars->mma_done[wg], mphase, abort_flag,
+                                                 status, kDevTimeoutAttn, TO);
+          mphase ^= 1;
+          // the Q buffer is free once the tile's last product is done: fetch the next one
+          const bool last_pass = (c0 + n >= i_t || ch == nchunks - 1) && p0 + C::PIECE >= n_t;
+          if (row == 0 && w && last_pass) {
+            const int t = next_scored(tile + 2);
+            if (t < ntiles) load_q(t);
+          }
+          if (__all_sync(0xffffffffu, w)) {
+            tc_fence_after();
+            for (int cc = 0; cc < np; cc += 32) {
+              uint32_t sr[32];
+              tmem_ld32(t_s + cc, sr);
+              tmem_wait_ld();
+#pragma unroll
+              for (int x = 0; x < 32; ++x) reg_fence(sr[x]);
+              // candidates: columns that beat this row's current threshold
+              const float thr0 = vals[KCAP - 1];
+              uint32_t mask = 0;
+#pragma unroll
+              for (int x = 0; x < 32; ++x) {
+                stage[x * 128 + row] = __uint_as_float(sr[x]);
+                if (cc + x < np && __uint_as_float(sr[x]) > thr0) mask |= 1u << x;
+              }
+              const int jb = c0 + p0 + cc;
+              while (__any_sync(0xffffffffu, mask != 0)) {
+                if (mask) {
+                  const int x = __ffs(mask) - 1;
+                  mask &= mask - 1;
+                  const float sc = stage[x * 128 + row];
+                  if (sc > vals[KCAP - 1]) insert_top<KCAP>(vals, ids, sc, jb + x);
+                }
+              }
+              __syncwarp();
+            }
+            tc_fence_before();
+          }
+          // every thread of the warpgroup has read the scores before the next pass overwrites them
+          ok = named_bar_and(1 + wg, 128, w);
+        }
+      }
+      if (!scored || row >= rows || !ok) continue;
+      int sel[KCAP];
+#pragma unroll
+      for (int x = 0; x < KCAP; ++x) sel[x] = (x < ksel) ? ids[x] : 0x7fffffff;
+#pragma unroll
+      for (int a0 = 0; a0 < KCAP - 1; ++a0) {
+#pragma unroll
+        for (int b0 = 0; b0 < KCAP - 1 - a0; ++b0) {
+          if (sel[b0] > sel[b0 + 1]) {
+            const int tmp = sel[b0];
+            sel[b0] = sel[b0 + 1];
+            sel[b0 + 1] = tmp;
+          }
+        }
+      }
+      int32_t* out = idx + (static_cast<size_t>(h) * T + t0 + row) * topk;
+#pragma unroll
+      for (int x = 0; x < KCAP; ++x)
+        if (x < ksel) out[x] = sel[x];
+      out[ksel] = i_t;
+    }
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+namespace {
+
+typedef CUresult (*EncodeTiledFnG)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool make_q_map(CUtensorMap* map, const void* q, int T, int H, int D) {
+  static EncodeTiledFnG fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) !=
+            cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess)
+      return false;
+    fn = reinterpret_cast<EncodeTiledFnG>(p);
+  }
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kTile)};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int KCAP>
+cudaError_t launch_t(const CUtensorMap& mq, const float* cents, const int32_t* cu, int nseq,
+                     int max_nb, int T, int H, int G, int B, int topk, int32_t* idx, int* status,
+                     int grid, cudaStream_t stream) {
+  const int smem = GateCfg<D>::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(gate_tc_kernel<D, KCAP>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  gate_tc_kernel<D, KCAP><<<grid, 256, smem, stream>>>(mq, cents, cu, nseq, max_nb, T, H, G, B,
+                                                       topk, idx, status);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const CUtensorMap& mq, const float* cents, const int32_t* cu, int nseq,
+                     int max_nb, int T, int H, int G, int B, int topk, int32_t* idx, int* status,
+                     int grid, cudaStream_t stream) {
+  const int ksel = topk - 1;
+  if (ksel <= 4) return launch_t<D, 4>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status, grid, stream);
+  if (ksel <= 8) return launch_t<D, 8>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status, grid, stream);
+  if (ksel <= 16) return launch_t<D, 16>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status, grid, stream);
+  return launch_t<D, 32>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status, grid, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_gate_tc(const void* q, const float* cents, const int32_t* cu_dev, int nseq,
+                           int max_nb, int T, int H, int G, int d, int B, int topk, int32_t* idx,
+                           int* status, int num_sms, cudaStream_t stream) {
+  if (topk - 1 > 32) return cudaErrorInvalidValue;
+  CUtensorMap mq;
+  if (!make_q_map(&mq, q, T, H, d)) return cudaErrorInvalidValue;
+  const int grid = num_sms > 0 ? num_sms : 1;  // persistent CTAs over the work units
+  if (d == 64)
+    return launch_d<64>(mq, cents, cu_dev, nseq, max_nb, T, H, G, B, topk, idx, status, grid, stream);
+  return launch_d<128>(mq, cents, cu_dev, nseq, max_nb, T, H, G, B, topk, idx, status, grid, stream);
+}
+
+}  // namespace moba

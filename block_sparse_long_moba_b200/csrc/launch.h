@@ -18,6 +18,11 @@ cudaError_t launch_gate(const void* q, const float* cents, const int32_t* cu_dev
                         int max_nb, int T, int H, int G, int d, int B, int topk, int32_t* idx,
                         cudaStream_t stream);
 
+// Tensor-core gate (scores on tcgen05, top-k in registers). `status` may be null.
+cudaError_t launch_gate_tc(const void* q, const float* cents, const int32_t* cu_dev, int nseq,
+                           int max_nb, int T, int H, int G, int d, int B, int topk, int32_t* idx,
+                           int* status, int num_sms, cudaStream_t stream);
+
 cudaError_t launch_route_count(const int32_t* idx, const BlockTables& tb, int T, int H, int G,
                                int topk, int NB, int b0, int nblk, int T0, int max_nb,
                                int* counts, cudaStream_t stream);

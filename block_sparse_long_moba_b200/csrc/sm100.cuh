@@ -257,6 +257,18 @@ __device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t nthreads, boo
   return r != 0;
 }
 
+// Barrier over `nthreads` threads that also returns the AND of `v` over them.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, %3, p;\n"
+      " selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 // -------------------------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor, 128-byte swizzle. lbo/sbo in bytes.
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {

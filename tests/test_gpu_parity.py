@@ -53,6 +53,8 @@ def test_centroids_match_oracle(moba, cu, hkv, d, B):
     ([0, 700, 700, 2000], 8, 2, 128, 64, 5, "offset"),
     ([0, 3000], 4, 4, 64, 64, 33, "clusters"),
     ([0, 2048], 2, 1, 128, 128, 1, "offset"),
+    ([0, 6144], 2, 2, 64, 64, 40, "clusters"),          # topk above the buffered-selection limit
+    ([0, 20000, 20000, 40000], 2, 1, 128, 64, 33, "clusters"),  # > 256 past blocks: chunked
 ])
 def test_gate_matches_oracle(moba, cu, hq, hkv, d, B, topk, keys):
     w, q, k, v, cu_t = _inputs(cu, hq, hkv, d, B, topk, keys)
