@@ -177,8 +177,8 @@ Layout layout_of(const Plan& P, int nseq, int Hq, int Hkv, int d, int topk) {
 template <class T>
 T* at(void* base, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(base) + off); }
 
-// The tensor-core gate buffers 64 candidates per row and keeps room for 32 new ones, so it serves
-// topk <= 33; larger topk uses the CUDA-core gate.
+// The tensor-core gate keeps at most 32 past blocks per row in registers, so it serves topk <= 33;
+// larger topk uses the CUDA-core gate.
 cudaError_t run_gate(const void* q, const float* cents, const int32_t* cu_dev, int nseq, int max_nb,
                      int T, int H, int G, int d, int B, int topk, int32_t* idx, int* status,
                      int sms, cudaStream_t s) {

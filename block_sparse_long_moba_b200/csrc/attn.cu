@@ -56,8 +56,8 @@ struct AttnArgs {
   float scale_log2;        // scale * log2(e)
 };
 
-struct Item {
-  int kind;  // 0 empty, 1 routed, 2 diagonal
+struct __align__(16) Item {
+  int kind;  // 0 empty, 1 routed, 2 diagonal, -1 end of the CTA's work
   int g, h, b;
   int key0, klen, nsub;
   int rows;     // valid rows of the item (<= 256)
@@ -108,55 +108,149 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, int w, int n_rout
   return it;
 }
 
-template <int D>
-struct AttnCfg {
-  static constexpr int NCB = D / 64;                  // 64-column (128-byte) swizzle blocks
-  static constexpr int HALF_BYTES = kTile * D * 2;    // one 128 x D bf16 tile
-  static constexpr int Q_BYTES = 2 * HALF_BYTES;      // one 256-row item
-  static constexpr int QB = (D == 128) ? 1 : 2;       // Q buffers
-  static constexpr int NST = (D == 128) ? 2 : 4;      // K and V ring depth
-  static constexpr int SMEM_TILES = QB * Q_BYTES + 2 * NST * HALF_BYTES;
-  static constexpr int SMEM_BYTES = SMEM_TILES + 1024 /*barriers*/ + 1024 /*alignment slack*/;
-  static constexpr uint32_t TMEM_COLS = 512;
-  // Registers per thread: launch budget (384 threads at 168) re-split between the control
-  // warpgroup (producer, MMA, gather) and the two softmax warpgroups; 128*72 + 256*216 = 384*168.
-  static constexpr uint32_t REGS_LAUNCH = 168, REGS_CTRL = 72, REGS_SOFTMAX = 216;
-  // TMEM columns: S/P of half x at 128 * x, O of half x at 256 + D * x
-  __host__ __device__ static constexpr uint32_t tm_s(int x) { return 128u * x; }
-  __host__ __device__ static constexpr uint32_t tm_o(int x) { return 256u + D * x; }
+// ------------------------------------------------------------------------------------------
+// Work-item ring. One scheduler warp decodes the CTA's work items 32 at a time (one per lane, so
+// the global loads of the routing tiles and block tables of 32 items overlap) and publishes the
+// non-empty ones, in order, into a small shared-memory ring, followed by an end marker. Every
+// other role copies each item out of the ring and frees the slot at once, so no role waits on a
+// global load to learn what to do next.
+constexpr int kRing = 16;
+
+struct ItemRing {
+  Item items[kRing];
+  uint64_t full[kRing], empty[kRing];
 };
 
-struct AttnBars {
-  uint64_t q_full[2], q_empty[2];
-  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full[2], p_full[2], o_full[2];
+// Scheduler side: one whole, converged warp. Returns false after an abort.
+__device__ __forceinline__ bool ring_produce(ItemRing* ring, const AttnArgs& a, int n_items,
+                                             int n_routed, volatile int* abort_flag, int* err,
+                                             uint64_t timeout_ns) {
+  const int lane = threadIdx.x & 31;
+  uint32_t n = 0;
+  auto publish = [&](const Item& it, int src) -> bool {
+    const uint32_t slot = n % kRing;
+    const bool ok = __all_sync(0xffffffffu,
+                               mbar_wait_bounded(&ring->empty[slot], ((n / kRing) & 1) ^ 1,
+                                                 abort_flag, err, kDevTimeoutAttn, timeout_ns));
+    if (!ok) return false;
+    if (lane == src) {
+      ring->items[slot] = it;
+      mbar_arrive(&ring->full[slot]);
+    }
+    ++n;
+    return true;
+  };
+  const int stride = static_cast<int>(gridDim.x);
+  for (int w0 = blockIdx.x; w0 < n_items; w0 += 32 * stride) {
+    const int w = w0 + lane * stride;
+    Item it;
+    it.kind = 0;
+    if (w < n_items) it = decode_item(a, w, n_routed);
+    uint32_t m = __ballot_sync(0xffffffffu, it.kind != 0);
+    while (m) {
+      const int src = __ffs(m) - 1;
+      m &= m - 1;
+      if (!publish(it, src)) return false;
+    }
+  }
+  Item end;
+  end.kind = -1;
+  end.g = end.h = end.b = end.key0 = end.klen = end.nsub = 0;
+  end.rows = end.start = end.qtok0 = end.qoff = end.slot = 0;
+  return publish(end, 0);
+}
+
+// True if item number `lt` has been published (does not wait).
+__device__ __forceinline__ bool ring_ready(ItemRing* ring, uint32_t lt) {
+  return mbar_try_wait(&ring->full[lt % kRing], (lt / kRing) & 1);
+}
+
+// Consumer side: copies item number `lt` of this CTA and frees its slot.
+__device__ __forceinline__ bool ring_consume(ItemRing* ring, uint32_t lt, Item& it,
+                                             volatile int* abort_flag, int* err,
+                                             uint64_t timeout_ns) {
+  const uint32_t slot = lt % kRing;
+  if (!mbar_wait_bounded(&ring->full[slot], (lt / kRing) & 1, abort_flag, err, kDevTimeoutAttn,
+                         timeout_ns))
+    return false;
+  it = ring->items[slot];
+  mbar_arrive(&ring->empty[slot]);
+  return true;
+}
+
+// ------------------------------------------------------------------------------------------
+// d = 64 kernel.
+//
+// Roles (384 threads): warp 0 = TMA producer of K/V sub-tiles; warp 1 = TMEM owner and MMA issuer
+// (the whole warp runs converged, elect.sync picks the issuing lane); warp 2 = Q row gather;
+// warp 3 = item scheduler; warps 4-7 = softmax and epilogue of half A; warps 8-11 = half B.
+//
+// Small blocks make small items (a 128-key block is one sub-tile), so the per-item overheads are
+// what this kernel is shaped around:
+//   * the gather first reads the item's routing entries with coalesced loads, then issues its
+//     16-byte row copies and keeps two items in flight (cp.async groups), QB items ahead;
+//   * O accumulators are double-buffered in TMEM per half (item parity), and the epilogue of an
+//     item runs after the next item's softmax, so it never delays the tensor pipe;
+//   * an item of at most 128 rows (every diagonal item of a 128-key block, the tail item of a
+//     routed list) runs on half A only: half B issues no MMA and its warps skip the item.
+struct D64Cfg {
+  static constexpr int D = 64;
+  static constexpr int HALF_BYTES = kTile * D * 2;  // 16 KB: one 128 x 64 bf16 tile
+  static constexpr int Q_BYTES = 2 * HALF_BYTES;    // one 256-row item
+  static constexpr int QB = 4;                      // Q buffers (items gathered ahead)
+  static constexpr int NST = 2;                     // K and V ring depth
+  static constexpr int OFF_K = QB * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NST * HALF_BYTES;
+  static constexpr int OFF_BARS = OFF_V + NST * HALF_BYTES;
+  static constexpr int SMEM_BYTES = OFF_BARS + 8192;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t REGS_CTRL = 72, REGS_SOFTMAX = 216;  // 128*72 + 256*216 = 384*168
+  static constexpr uint32_t RING_CONSUMERS = 3 * 32 + 256;       // warps 0-2 and the softmax
+  // TMEM columns: S/P of half x at 128 x; O of half x for item parity p at 256 + 64 (2 p + x)
+  __host__ __device__ static constexpr uint32_t tm_s(int x) { return 128u * x; }
+  __host__ __device__ static constexpr uint32_t tm_o(int x, uint32_t p) {
+    return 256u + 64u * (2u * p + static_cast<uint32_t>(x));
+  }
+};
+static_assert(D64Cfg::SMEM_BYTES <= 232448, "shared memory budget of one CTA");
+
+struct D64Bars {
+  uint64_t q_full[D64Cfg::QB], q_empty[D64Cfg::QB];
+  uint64_t k_full[D64Cfg::NST], k_empty[D64Cfg::NST], v_full[D64Cfg::NST], v_empty[D64Cfg::NST];
+  uint64_t s_full[2], p_full[2], o_full[2][2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
+  ItemRing ring;
+  int q_row[kItemRows];  // gather scratch: query row (t * H + h) of each item row, -1 = none
+  // per softmax thread: the previous item's output row (-1 = none), 1 / l and log-sum-exp
+  int ep_row[kItemRows];
+  float ep_inv[kItemRows], ep_lse[kItemRows];
 };
+static_assert(sizeof(D64Bars) <= 8192, "barrier block");
 
-template <int D>
 __global__ void __launch_bounds__(384, 1)
-    attn_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
-                const AttnArgs a) {
-  using C = AttnCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;                              // [QB][2 halves][NCB][16 KB]
-  uint8_t* sK = sQ + C::QB * C::Q_BYTES;           // [NST][NCB][16 KB]
-  uint8_t* sV = sK + C::NST * C::HALF_BYTES;       // [NST][NCB][16 KB]
-  AttnBars* bars = reinterpret_cast<AttnBars*>(sV + C::NST * C::HALF_BYTES);
+    attn_kernel_d64(const __grid_constant__ CUtensorMap map_k,
+                    const __grid_constant__ CUtensorMap map_v, const AttnArgs a) {
+  using C = D64Cfg;
+  constexpr int D = C::D;
+  extern __shared__ __align__(1024) uint8_t smem64[];
+  uint8_t* sQ = smem64;
+  uint8_t* sK = smem64 + C::OFF_K;
+  uint8_t* sV = smem64 + C::OFF_V;
+  D64Bars* bars = reinterpret_cast<D64Bars*>(smem64 + C::OFF_BARS);
+  ItemRing* ring = &bars->ring;
   volatile int* abort_flag = &bars->abort_flag;
-
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the swizzled layouts assume a 1024-byte aligned base: refuse to run otherwise
+  if (smem_u32(smem64) & 1023u) {
+    if (tid == 0) atomicCAS(a.status, 0, kDevTimeoutAttn);
+    return;
+  }
   if (tid == 0) {
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(&bars->q_full[x], 64);
+    for (int x = 0; x < C::QB; ++x) {
+      mbar_init(&bars->q_full[x], 32);
       mbar_init(&bars->q_empty[x], 1);
-      mbar_init(&bars->s_full[x], 1);
-      mbar_init(&bars->p_full[x], 128);
-      mbar_init(&bars->o_full[x], 1);
     }
     for (int x = 0; x < C::NST; ++x) {
       mbar_init(&bars->k_full[x], 1);
@@ -164,7 +258,17 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->v_full[x], 1);
       mbar_init(&bars->v_empty[x], 1);
     }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->p_full[x], 128);
+      mbar_init(&bars->o_full[x][0], 1);
+      mbar_init(&bars->o_full[x][1], 1);
+    }
     mbar_init(&bars->drain, 1);
+    for (int x = 0; x < kRing; ++x) {
+      mbar_init(&ring->full[x], 1);
+      mbar_init(&ring->empty[x], C::RING_CONSUMERS);
+    }
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -180,23 +284,24 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-
   const int n_routed = *a.n_routed;
   const int n_items = n_routed + a.n_diag;
   const uint64_t TO = kWaitTimeoutNs;
   int* err = a.status;
+  auto pop = [&](uint32_t lt, Item& it) -> bool {
+    return ring_consume(ring, lt, it, abort_flag, err, TO);
+  };
 
   if (warp < 4) {
-   regs_dec<C::REGS_CTRL>();
-   if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer (K, V)
-    // The whole warp runs the loop (converged); elect.sync picks the issuing lane.
-    {
+    regs_dec<C::REGS_CTRL>();
+    if (warp == 0) {
+      // -------------------------------------------------------------- TMA producer (K, V)
       uint32_t J = 0, issued_k = 0, issued_v = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
-        const Item it = decode_item(a, w, n_routed);
-        if (it.kind == 0) continue;
+      for (uint32_t lt = 0;; ++lt) {
+        Item it;
+        ok = __all_sync(0xffffffffu, pop(lt, it));
+        if (!ok || it.kind < 0) break;
         for (int j = 0; j < it.nsub; ++j, ++J) {
           const int st = J % C::NST;
           const uint32_t ph = (J / C::NST) & 1;
@@ -205,21 +310,16 @@ __global__ void __launch_bounds__(384, 1)
                                                          err, kDevTimeoutAttn, TO));
           if (!ok) break;
           mbar_arrive_expect_tx_elect(&bars->k_full[st], C::HALF_BYTES);
-#pragma unroll
-          for (int c = 0; c < C::NCB; ++c)
-            tma_load_3d_elect(sK + st * C::HALF_BYTES + c * 16384, &map_k, &bars->k_full[st],
-                              c * 64, it.g, tok);
+          tma_load_3d_elect(sK + st * C::HALF_BYTES, &map_k, &bars->k_full[st], 0, it.g, tok);
           ++issued_k;
           ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->v_empty[st], ph ^ 1, abort_flag,
                                                          err, kDevTimeoutAttn, TO));
           if (!ok) break;
           mbar_arrive_expect_tx_elect(&bars->v_full[st], C::HALF_BYTES);
-#pragma unroll
-          for (int c = 0; c < C::NCB; ++c)
-            tma_load_3d_elect(sV + st * C::HALF_BYTES + c * 16384, &map_v, &bars->v_full[st],
-                              c * 64, it.g, tok);
+          tma_load_3d_elect(sV + st * C::HALF_BYTES, &map_v, &bars->v_full[st], 0, it.g, tok);
           ++issued_v;
         }
+        if (!ok) break;
       }
       if (!ok) {
         // after an abort, let the loads still in flight land before the CTA exits (bounded)
@@ -227,68 +327,64 @@ __global__ void __launch_bounds__(384, 1)
         for (uint32_t x = 0; x < static_cast<uint32_t>(C::NST); ++x) {
           if (issued_k > x) {
             const uint32_t Jx = issued_k - 1 - x;
-            mbar_wait_bounded(&bars->k_full[Jx % C::NST], (Jx / C::NST) & 1, &no_abort, nullptr, 0, TO / 4);
+            mbar_wait_bounded(&bars->k_full[Jx % C::NST], (Jx / C::NST) & 1, &no_abort, nullptr,
+                              0, TO / 4);
           }
           if (issued_v > x) {
             const uint32_t Jx = issued_v - 1 - x;
-            mbar_wait_bounded(&bars->v_full[Jx % C::NST], (Jx / C::NST) & 1, &no_abort, nullptr, 0, TO / 4);
+            mbar_wait_bounded(&bars->v_full[Jx % C::NST], (Jx / C::NST) & 1, &no_abort, nullptr,
+                              0, TO / 4);
           }
         }
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------------ MMA issuer
-    // The whole warp runs the loop (converged, warp-uniform descriptors); elect.sync picks the
-    // lane that issues each tcgen05.mma / commit.
-    {
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-      uint32_t J = 0, lt = 0;
+      uint32_t J = 0;                // K/V sub-tiles consumed
+      uint32_t cs[2] = {0u, 0u};     // sub-tiles processed by each half (s_full / p_full phase)
+      uint32_t ci[2] = {0u, 0u};     // items processed by each half (O buffer, o_full)
       bool ok = true;
       auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
         return __all_sync(0xffffffffu,
                           mbar_wait_bounded(bar, parity, abort_flag, err, kDevTimeoutAttn, TO));
       };
       auto issue_s = [&](int half, uint32_t qb, int st) {
-        const uint32_t t_s = tmem + C::tm_s(half);
-        const uint32_t qbase = sQa + qb * C::Q_BYTES + half * C::HALF_BYTES;
+        const uint64_t ad = smem_desc_sw128(sQa + qb * C::Q_BYTES + half * C::HALF_BYTES, 16, 1024);
+        const uint64_t bd = smem_desc_sw128(sKa + st * C::HALF_BYTES, 16, 1024);
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          const uint64_t ad = smem_desc_sw128(qbase + off, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sKa + st * C::HALF_BYTES + off, 16, 1024);
-          mma_ss_elect(t_s, ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_ss_elect(tmem + C::tm_s(half), desc_advance(ad, ks * 32), desc_advance(bd, ks * 32),
+                       IDESC_QK, ks > 0 ? 1u : 0u);
         mma_commit_elect(&bars->s_full[half]);
       };
-      // O_x += P_x V_st; waits for P_x of sub-tile Jp
-      auto issue_pv = [&](int half, uint32_t Jp, bool first, bool last) -> bool {
-        const int st = Jp % C::NST;
-        if (!wait(&bars->p_full[half], Jp & 1)) return false;
+      // O_x += P_x V_st for the half's sub-tile number c of its item number item
+      auto issue_pv = [&](int half, int st, uint32_t c, uint32_t item, bool first, bool last,
+                          bool free_v) -> bool {
+        if (!wait(&bars->p_full[half], c & 1)) return false;
         tc_fence_after();
-        const uint32_t t_o = tmem + C::tm_o(half);
+        const uint32_t t_o = tmem + C::tm_o(half, item & 1);
         const uint32_t t_p = tmem + C::tm_s(half);
+        const uint64_t bd = smem_desc_sw128(sVa + st * C::HALF_BYTES, 16384, 1024);
 #pragma unroll
-        for (int ks = 0; ks < kTile / 16; ++ks) {
-          const uint64_t bd = smem_desc_sw128(sVa + st * C::HALF_BYTES + ks * 2048, 16384, 1024);
-          mma_ts_elect(t_o, t_p + ks * 8, bd, IDESC_PV, (first && ks == 0) ? 0u : 1u);
-        }
-        if (half == 1) mma_commit_elect(&bars->v_empty[st]);
-        if (last) mma_commit_elect(&bars->o_full[half]);
+        for (int ks = 0; ks < kTile / 16; ++ks)
+          mma_ts_elect(t_o, t_p + ks * 8, desc_advance(bd, ks * 2048), IDESC_PV,
+                       (first && ks == 0) ? 0u : 1u);
+        if (free_v) mma_commit_elect(&bars->v_empty[st]);
+        if (last) mma_commit_elect(&bars->o_full[half][item & 1]);
         return true;
       };
+      // PV of half B is issued one step late, after the next S of half A (ping-pong)
       bool pend = false, pend_first = false, pend_last = false;
-      uint32_t pend_J = 0;
-      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
-        const Item it = decode_item(a, w, n_routed);
-        if (it.kind == 0) continue;
+      int pend_st = 0;
+      uint32_t pend_c = 0, pend_item = 0;
+      for (uint32_t lt = 0;; ++lt) {
+        Item it;
+        ok = __all_sync(0xffffffffu, pop(lt, it));
+        if (!ok || it.kind < 0) break;
+        const bool hasB = it.rows > kTile;
         const uint32_t qb = lt % C::QB;
-        if (C::QB == 1 && pend) {  // a single Q buffer: finish the previous item first
-          ok = issue_pv(1, pend_J, pend_first, pend_last);
-          pend = false;
-          if (!ok) break;
-        }
         ok = wait(&bars->q_full[qb], (lt / C::QB) & 1);
         if (!ok) break;
         tc_fence_after();
@@ -299,72 +395,108 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
           issue_s(0, qb, st);
           if (pend) {
-            ok = issue_pv(1, pend_J, pend_first, pend_last);
             pend = false;
+            ok = issue_pv(1, pend_st, pend_c, pend_item, pend_first, pend_last, true);
             if (!ok) break;
           }
-          issue_s(1, qb, st);
+          if (hasB) issue_s(1, qb, st);
           mma_commit_elect(&bars->k_empty[st]);
           if (j == it.nsub - 1) mma_commit_elect(&bars->q_empty[qb]);
           ok = wait(&bars->v_full[st], (J / C::NST) & 1);
           if (!ok) break;
-          ok = issue_pv(0, J, j == 0, j == it.nsub - 1);
+          ok = issue_pv(0, st, cs[0], ci[0], j == 0, j == it.nsub - 1, !hasB);
           if (!ok) break;
-          pend = true;
-          pend_J = J;
-          pend_first = (j == 0);
-          pend_last = (j == it.nsub - 1);
+          ++cs[0];
+          if (hasB) {
+            pend = true;
+            pend_st = st;
+            pend_c = cs[1]++;
+            pend_item = ci[1];
+            pend_first = (j == 0);
+            pend_last = (j == it.nsub - 1);
+          }
         }
-        ++lt;
+        if (!ok) break;
+        ++ci[0];
+        if (hasB) ++ci[1];
       }
-      if (ok && pend) ok = issue_pv(1, pend_J, pend_first, pend_last);
+      if (ok && pend) ok = issue_pv(1, pend_st, pend_c, pend_item, pend_first, pend_last, true);
       if (!ok) {
         // after an abort, wait (bounded) until the MMAs already issued have finished with TMEM
         volatile int no_abort = 0;
         mma_commit_elect(&bars->drain);
         mbar_wait_bounded(&bars->drain, 0, &no_abort, nullptr, 0, TO / 4);
       }
-    }
-  } else if (warp < 4) {
-    // -------------------------------------------------------------------- Q row gather
-    const int gt = tid - 64;  // 0..63
-    constexpr int CPR = D / 8;  // 16-byte chunks per row
-    uint32_t lt = 0;
-    bool ok = true;
-    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
-      const Item it = decode_item(a, w, n_routed);
-      if (it.kind == 0) continue;
-      const uint32_t qb = lt % C::QB;
-      ok = mbar_wait_bounded(&bars->q_empty[qb], ((lt / C::QB) & 1) ^ 1, abort_flag, err, kDevTimeoutAttn, TO);
-      if (!ok) break;
-      const uint32_t dst0 = smem_u32(sQ + qb * C::Q_BYTES);
-      for (int e = gt; e < kItemRows * CPR; e += 64) {
-        const int m = e / CPR, c = e % CPR;
-        const __nv_bfloat16* src = a.q;
-        uint32_t bytes = 0;
-        if (m < it.rows) {
-          int t, h;
-          if (it.kind == 1) {
-            const int pr = __ldg(a.entries + it.start + m);
-            t = a.T0 + pr / (a.H * a.topk);
-            h = (pr / a.topk) % a.H;
-          } else {
-            t = it.qtok0 + m;
-            h = it.h;
-          }
-          src = a.q + (static_cast<size_t>(t) * a.H + h) * D + c * 8;
-          bytes = 16;
+    } else if (warp == 2) {
+      // ------------------------------------------------------------------ Q row gather
+      // Item rows are spread 4 per warp instruction (8 lanes x 16 bytes = one 128-byte row), so
+      // every copy instruction moves four whole rows.
+      const uint32_t sQa = smem_u32(sQ);
+      int* q_row = bars->q_row;
+      bool ok = true, pending = false;
+      uint32_t prev_qb = 0;
+      for (uint32_t lt = 0;; ++lt) {
+        const uint32_t qb = lt % C::QB;
+        const uint32_t par = ((lt / C::QB) & 1) ^ 1;
+        // publish the previous item first whenever the next one cannot start at once (keeps the
+        // MMA fed, and no wait below ever holds back an item the other roles need)
+        if (pending && !__all_sync(0xffffffffu, ring_ready(ring, lt) &&
+                                                    mbar_try_wait(&bars->q_empty[qb], par))) {
+          cp_async_wait_group<0>();
+          fence_proxy_async_smem();
+          mbar_arrive(&bars->q_full[prev_qb]);
+          pending = false;
         }
-        const uint32_t dst = dst0 + (m >> 7) * C::HALF_BYTES + (c >> 3) * 16384 +
-                             sw128_offset(m & 127, (c & 7) * 8);
-        cp_async_16(dst, src, bytes);
+        Item it;
+        ok = __all_sync(0xffffffffu, pop(lt, it));
+        if (!ok || it.kind < 0) break;
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->q_empty[qb], par, abort_flag, err,
+                                                       kDevTimeoutAttn, TO));
+        if (!ok) break;
+        // query row of every item row; the routing entries are read with coalesced loads first
+        int ent[kItemRows / 32];
+#pragma unroll
+        for (int u = 0; u < kItemRows / 32; ++u) {
+          const int m = lane + 32 * u;
+          ent[u] = (it.kind == 1 && m < it.rows) ? __ldg(a.entries + it.start + m) : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < kItemRows / 32; ++u) {
+          const int m = lane + 32 * u;
+          int qr = -1;
+          if (m < it.rows)
+            qr = (it.kind == 1) ? a.T0 * a.H + ent[u] / a.topk : (it.qtok0 + m) * a.H + it.h;
+          q_row[m] = qr;
+        }
+        __syncwarp();
+        const int nrows = it.rows > kTile ? kItemRows : kTile;
+        const uint32_t dst0 = sQa + qb * C::Q_BYTES;
+        const int c = lane & 7;
+        for (int m = lane >> 3; m < nrows; m += 4) {
+          const int qr = q_row[m];
+          const __nv_bfloat16* src = (qr >= 0) ? a.q + static_cast<size_t>(qr) * D + c * 8 : a.q;
+          const uint32_t dst = dst0 + (m >> 7) * C::HALF_BYTES + sw128_offset(m & 127, c * 8);
+          cp_async_16(dst, src, qr >= 0 ? 16u : 0u);
+        }
+        __syncwarp();
+        cp_async_commit();
+        if (pending) {
+          cp_async_wait_group<1>();
+          fence_proxy_async_smem();
+          mbar_arrive(&bars->q_full[prev_qb]);
+        }
+        pending = true;
+        prev_qb = qb;
       }
       cp_async_wait_all();
-      fence_proxy_async_smem();
-      mbar_arrive(&bars->q_full[qb]);
-      ++lt;
+      if (ok && pending) {
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->q_full[prev_qb]);
+      }
+    } else {
+      // ------------------------------------------------------------------ item scheduler
+      ring_produce(ring, a, n_items, n_routed, abort_flag, err, TO);
     }
-   }
   } else {
     regs_inc<C::REGS_SOFTMAX>();
     // ------------------------------------------------------------ softmax + epilogue
@@ -372,14 +504,50 @@ __global__ void __launch_bounds__(384, 1)
     const int row = tid - 128 - half * 128;  // TMEM lane / row inside the half
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t t_s = tmem + lane_off + C::tm_s(half);
-    const uint32_t t_o = tmem + lane_off + C::tm_o(half);
     const float sl2 = a.scale_log2;
-    uint32_t J = 0, lt = 0;
+    const int q = half * kTile + row;        // row inside the 256-row item
+    uint32_t cs = 0, ci = 0;  // sub-tiles and items processed by this half
     bool ok = true;
-    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
-      const Item it = decode_item(a, w, n_routed);
-      if (it.kind == 0) continue;
-      const int r_item = half * kTile + row;  // row inside the 256-row item
+    // epilogue of this half's item number ci - 1 (its output row, 1 / l and log-sum-exp are
+    // parked in shared memory meanwhile, to keep registers for the softmax)
+    auto epilogue = [&]() -> bool {
+      const uint32_t pci = ci - 1, ob = pci & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars->o_full[half][ob], (pci >> 1) & 1,
+                                                     abort_flag, err, kDevTimeoutAttn, TO)))
+        return false;
+      tc_fence_after();
+      const uint32_t t_o = tmem + lane_off + C::tm_o(half, ob);
+      const int prev_prow = bars->ep_row[q];
+      const bool prev_valid = prev_prow >= 0;
+      const float inv = bars->ep_inv[q];
+      uint4* dst = reinterpret_cast<uint4*>(a.part_o + static_cast<size_t>(prev_prow) * D);
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t orr[32];
+        tmem_ld32(t_o + c0, orr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) reg_fence(orr[x]);
+        if (prev_valid) {
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+            dst[c0 / 8 + x] = make_uint4(
+                pack_bf16x2(__uint_as_float(orr[8 * x + 0]) * inv, __uint_as_float(orr[8 * x + 1]) * inv),
+                pack_bf16x2(__uint_as_float(orr[8 * x + 2]) * inv, __uint_as_float(orr[8 * x + 3]) * inv),
+                pack_bf16x2(__uint_as_float(orr[8 * x + 4]) * inv, __uint_as_float(orr[8 * x + 5]) * inv),
+                pack_bf16x2(__uint_as_float(orr[8 * x + 6]) * inv, __uint_as_float(orr[8 * x + 7]) * inv));
+        }
+      }
+      tc_fence_before();
+      if (prev_valid) a.part_lse[prev_prow] = bars->ep_lse[q];
+      return true;
+    };
+    for (uint32_t lt = 0;; ++lt) {
+      Item it;
+      ok = __all_sync(0xffffffffu, pop(lt, it));
+      if (!ok || it.kind < 0) break;
+      if (half == 1 && it.rows <= kTile) continue;  // half B idle for this item
+      const int r_item = q;
       const bool valid = r_item < it.rows;
       int prow = 0, limit;
       if (it.kind == 1) {
@@ -390,10 +558,11 @@ __global__ void __launch_bounds__(384, 1)
         prow = ((t - a.T0) * a.H + it.h) * a.topk + it.slot;
         limit = valid ? it.qoff + r_item + 1 : 1;
       }
+      const uint32_t t_o = tmem + lane_off + C::tm_o(half, ci & 1);
       float m_ref = -INFINITY, l_sum = 0.f;
-      for (int j = 0; j < it.nsub; ++j, ++J) {
-        ok = mbar_wait_bounded(&bars->s_full[half], J & 1, abort_flag, err, kDevTimeoutAttn, TO);
-        ok = __all_sync(0xffffffffu, ok);
+      for (int j = 0; j < it.nsub; ++j, ++cs) {
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[half], cs & 1, abort_flag,
+                                                       err, kDevTimeoutAttn, TO));
         if (!ok) break;
         tc_fence_after();
         uint32_t sr[128];
@@ -469,7 +638,6 @@ __global__ void __launch_bounds__(384, 1)
           for (int x = 0; x < 8; ++x) {
             const float t0 = fmaf(__uint_as_float(sr[c + 2 * x]), sl2, neg);
             const float t1 = fmaf(__uint_as_float(sr[c + 2 * x + 1]), sl2, neg);
-            // kPolyPairs of every 8 column pairs go to the FMA pipe, the rest to MUFU.EX2
             const bool poly = x >= 8 - kPolyPairs;
             const float p0 = poly ? exp2_poly(t0) : ex2_approx(t0);
             const float p1 = poly ? exp2_poly(t1) : ex2_approx(t1);
@@ -485,34 +653,17 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive(&bars->p_full[half]);
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16 partial row, log-sum-exp
-      ok = mbar_wait_bounded(&bars->o_full[half], lt & 1, abort_flag, err, kDevTimeoutAttn, TO);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      const float inv = 1.f / l_sum;
-      __nv_bfloat16* dst = a.part_o + static_cast<size_t>(prow) * D;
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t orr[32];
-        tmem_ld32(t_o + c0, orr);
-        tmem_wait_ld();
-#pragma unroll
-        for (int x = 0; x < 32; ++x) reg_fence(orr[x]);
-        if (valid) {
-          uint4 pkt[4];
-          uint32_t* pw = reinterpret_cast<uint32_t*>(pkt);
-#pragma unroll
-          for (int x = 0; x < 16; ++x)
-            pw[x] = pack_bf16x2(__uint_as_float(orr[2 * x]) * inv, __uint_as_float(orr[2 * x + 1]) * inv);
-#pragma unroll
-          for (int x = 0; x < 4; ++x) reinterpret_cast<uint4*>(dst + c0)[x] = pkt[x];
-        }
+      // the previous item's O is complete by now (its last PV preceded this item's S)
+      if (ci > 0) {
+        ok = epilogue();
+        if (!ok) break;
       }
-      if (valid) a.part_lse[prow] = (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
-      tc_fence_before();
-      ++lt;
+      bars->ep_row[q] = valid ? prow : -1;
+      bars->ep_inv[q] = 1.f / l_sum;
+      bars->ep_lse[q] = (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
+      ++ci;
     }
+    if (ok && ci > 0) ok = epilogue();
   }
 
   tc_fence_before();
@@ -551,7 +702,8 @@ struct PvtCfg {
   static constexpr int SMEM_BYTES = OFF_BARS + 256;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t TM_OT = 256;
-  static constexpr uint32_t REGS_CTRL = 72, REGS_SOFTMAX = 216;
+  // the MMA issuer needs ~100 registers; 128*104 + 256*200 = 384*168 leaves nothing spilled
+  static constexpr uint32_t REGS_CTRL = 104, REGS_SOFTMAX = 200;
   __host__ __device__ static constexpr uint32_t tm_s(int x) { return 128u * x; }
 };
 static_assert(PvtCfg::SMEM_BYTES <= 232448, "shared memory budget of one CTA");
@@ -705,12 +857,12 @@ __global__ void __launch_bounds__(384, 1)
         if (J > 0 && !wait(&bars->s_free[x], (J - 1) & 1)) return false;
         tc_fence_after();
         const int st = J & 1;
-        const uint32_t qbase = sQa + x * C::HALF_BYTES;
+        const uint64_t ad = smem_desc_sw128(sQa + x * C::HALF_BYTES, 16, 1024);
+        const uint64_t bd = smem_desc_sw128(sKa + st * C::HALF_BYTES, 16, 1024);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_ss_elect(tmem + C::tm_s(x), smem_desc_sw128(qbase + off, 16, 1024),
-                       smem_desc_sw128(sKa + st * C::HALF_BYTES + off, 16, 1024), IDESC_QK,
+          mma_ss_elect(tmem + C::tm_s(x), desc_advance(ad, off), desc_advance(bd, off), IDESC_QK,
                        ks > 0 ? 1u : 0u);
         }
         mma_commit_elect(&bars->s_full[x]);
@@ -729,12 +881,13 @@ __global__ void __launch_bounds__(384, 1)
         if (!wait(&bars->v_full, J & 1)) return false;
         if (!wait(&bars->p_full, J & 1)) return false;
         tc_fence_after();
+        const uint64_t ad = smem_desc_sw128(sVa, 16384, 1024);
+        const uint64_t bd = smem_desc_sw128(sPa, 16, 1024);
 #pragma unroll
-        for (int ks = 0; ks < kTile / 16; ++ks) {
-          const uint64_t ad = smem_desc_sw128(sVa + ks * 2048, 16384, 1024);
-          const uint64_t bd = smem_desc_sw128(sPa + (ks >> 2) * 32768 + (ks & 3) * 32, 16, 1024);
-          mma_ss_elect(tmem + C::TM_OT, ad, bd, IDESC_PVT, (first && ks == 0) ? 0u : 1u);
-        }
+        for (int ks = 0; ks < kTile / 16; ++ks)
+          mma_ss_elect(tmem + C::TM_OT, desc_advance(ad, ks * 2048),
+                       desc_advance(bd, (ks >> 2) * 32768 + (ks & 3) * 32), IDESC_PVT,
+                       (first && ks == 0) ? 0u : 1u);
         mma_commit_elect(&bars->v_empty);
         mma_commit_elect(&bars->pv_done);
         return true;
@@ -1030,17 +1183,18 @@ cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream) {
   // setmaxnreg.inc would wait forever if the launch had fewer registers than the split assumes
   {
     cudaFuncAttributes fa;
-    cudaError_t e = (L.d == 64) ? cudaFuncGetAttributes(&fa, attn_kernel<64>)
+    cudaError_t e = (L.d == 64) ? cudaFuncGetAttributes(&fa, attn_kernel_d64)
                                 : cudaFuncGetAttributes(&fa, attn_kernel_pvt);
     if (e != cudaSuccess) return e;
-    const int need = 128 * AttnCfg<128>::REGS_CTRL + 256 * AttnCfg<128>::REGS_SOFTMAX;
+    const int need = (L.d == 64) ? 128 * D64Cfg::REGS_CTRL + 256 * D64Cfg::REGS_SOFTMAX
+                                 : 128 * PvtCfg::REGS_CTRL + 256 * PvtCfg::REGS_SOFTMAX;
     if (fa.numRegs * 384 < need) return cudaErrorInvalidConfiguration;
   }
   if (L.d == 64) {
-    const int smem = AttnCfg<64>::SMEM_BYTES;
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int smem = D64Cfg::SMEM_BYTES;
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel_d64, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_kernel<64><<<grid, 384, smem, stream>>>(mk, mv, a);
+    attn_kernel_d64<<<grid, 384, smem, stream>>>(mk, mv, a);
   } else {
     const int smem = PvtCfg::SMEM_BYTES;
     cudaError_t e = cudaFuncSetAttribute(attn_kernel_pvt, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -10,9 +10,12 @@
 //
 // Selection: one thread per row (= TMEM lane) keeps its running top list in registers, sorted
 // best first (strict comparison, so equal scores keep the lower block). Scores are read 32 at a
-// time, staged in shared memory, and each row visits only the columns that beat its current
-// threshold, so a warp pays for the largest per-row candidate count of a chunk rather than for
-// every column.
+// time; only when some row of the warp has a column that beats its current threshold are they
+// staged in shared memory, and each row then visits only those columns, so a warp pays for the
+// largest per-row candidate count of a chunk rather than for every column. An insertion computes
+// every position of the list independently (no compare-and-swap chain), so its cost is issue
+// slots rather than latency. Scores live in two 128-column TMEM buffers per warpgroup: the
+// products of the next 128 past blocks run on the tensor core while this piece is selected.
 //
 // A CTA holds two warpgroups (one query tile each) and works on one (query block, kv head) unit at a
 // time: the split centroids of the unit's past blocks are converted into shared memory once and
@@ -37,13 +40,13 @@ struct GateCfg {
   static constexpr int OFF_STAGE = OFF_B + B_BYTES;          // [2][32][128] staged scores
   static constexpr int OFF_BARS = OFF_STAGE + 2 * 32 * 128 * 4;
   static constexpr int SMEM_BYTES = OFF_BARS + 256;
-  static constexpr int PIECE = 256;                          // MMA N (scores per TMEM pass)
+  static constexpr int PIECE = 128;                          // MMA N (scores per TMEM buffer)
 };
 static_assert(GateCfg<128>::SMEM_BYTES <= 232448 && GateCfg<64>::SMEM_BYTES <= 232448,
               "shared memory budget of one CTA");
 
 struct GateBars {
-  uint64_t q_full[2], mma_done[2];
+  uint64_t q_full[2], mma_done[2][2];
   uint32_t tmem_base;
   int abort_flag;
   int red[32];
@@ -56,21 +59,21 @@ __device__ __forceinline__ uint32_t c_offset(int s, int row, int col) {
          sw128_offset(row, col & 63);
 }
 
+// Inserts (s, j) into the list sorted best first; requires s > vals[KCAP - 1]. An entry equal to s
+// stays ahead of it. gt[] is monotone (the list is sorted), so position x takes the entry above it
+// when s beats that one, s when s beats only the entry at x, and keeps its entry otherwise.
 template <int KCAP>
 __device__ __forceinline__ void insert_top(float (&vals)[KCAP], int (&ids)[KCAP], float s, int j) {
-  vals[KCAP - 1] = s;
-  ids[KCAP - 1] = j;
+  bool gt[KCAP];
+#pragma unroll
+  for (int x = 0; x < KCAP; ++x) gt[x] = s > vals[x];
 #pragma unroll
   for (int x = KCAP - 1; x > 0; --x) {
-    if (vals[x] > vals[x - 1]) {
-      const float tv = vals[x];
-      vals[x] = vals[x - 1];
-      vals[x - 1] = tv;
-      const int ti = ids[x];
-      ids[x] = ids[x - 1];
-      ids[x - 1] = ti;
-    }
+    vals[x] = gt[x - 1] ? vals[x - 1] : (gt[x] ? s : vals[x]);
+    ids[x] = gt[x - 1] ? ids[x - 1] : (gt[x] ? j : ids[x]);
   }
+  vals[0] = gt[0] ? s : vals[0];
+  ids[0] = gt[0] ? j : ids[0];
 }
 
 }  // namespace
@@ -93,7 +96,8 @@ __global__ void __launch_bounds__(256, 1)
   if (tid == 0) {
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->q_full[x], 1);
-      mbar_init(&bars->mma_done[x], 1);
+      mbar_init(&bars->mma_done[x][0], 1);
+      mbar_init(&bars->mma_done[x][1], 1);
     }
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -107,14 +111,15 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const uint32_t t_s = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + wg * C::PIECE;
+  const uint32_t t_s = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + wg * 2 * C::PIECE;
   uint8_t* sQ = smem + wg * C::Q_BYTES;
   float* stage = reinterpret_cast<float*>(smem + C::OFF_STAGE) + wg * 32 * 128;  // [x][row]
   const uint32_t sBa = smem_u32(smem + C::OFF_B);
   const int r = H / G;
   const int ksel = topk - 1;
   const uint64_t TO = kWaitTimeoutNs;
-  uint32_t qphase = 0, mphase = 0;  // barrier phases of this warpgroup
+  uint32_t qphase = 0;  // q_full phase of this warpgroup
+  uint32_t npiece = 0;  // score pieces issued by this warpgroup (TMEM buffer npiece & 1)
   bool ok = true;
 
   // Work units: (sequence, kv head g, group of QG consecutive query blocks, sub-range of at most
@@ -246,32 +251,41 @@ __global__ void __launch_bounds__(256, 1)
           q_ready = true;
           ok = named_bar_and(1 + wg, 128, w);
         }
-        // scores of this chunk in passes of up to 256 blocks
+        // scores of this chunk, 128 past blocks per TMEM buffer; the products of piece p + 1 are
+        // issued before piece p is selected (its buffer was freed by the barrier ending p - 1)
+        const uint32_t qa = smem_u32(sQ);
+        auto issue = [&](int p0) {  // one converged warp of the warpgroup issues
+          const int nmma = (min(C::PIECE, n_t - p0) + 15) & ~15;
+          const uint32_t idesc = idesc_bf16_f32(128, nmma, 0, 0);
+          const uint32_t buf = npiece & 1;
+          tc_fence_after();
+#pragma unroll
+          for (int sp = 0; sp < 2; ++sp) {
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint32_t aoff = (ks >> 2) * 16384 + (ks & 3) * 32;
+              const uint32_t boff = static_cast<uint32_t>(sp * C::NCB * C::CAP * 128 +
+                                                          (ks >> 2) * C::CAP * 128 + p0 * 128 +
+                                                          (ks & 3) * 32);
+              mma_ss_elect(tmem + wg * 2 * C::PIECE + buf * C::PIECE,
+                           smem_desc_sw128(qa + aoff, 16, 1024),
+                           smem_desc_sw128(sBa + boff, 16, 1024), idesc,
+                           (sp > 0 || ks > 0) ? 1u : 0u);
+            }
+          }
+          mma_commit_elect(&bars->mma_done[wg][buf]);
+        };
+        if (ok && warp == wg * 4) issue(0);
+        ++npiece;
         for (int p0 = 0; p0 < n_t; p0 += C::PIECE) {
           const int np = min(C::PIECE, n_t - p0);
-          const int nmma = (np + 15) & ~15;
-          if (ok && warp == wg * 4) {  // one converged warp of the warpgroup issues
-            tc_fence_after();
-            const uint32_t idesc = idesc_bf16_f32(128, nmma, 0, 0);
-            const uint32_t qa = smem_u32(sQ);
-#pragma unroll
-            for (int sp = 0; sp < 2; ++sp) {
-#pragma unroll
-              for (int ks = 0; ks < D / 16; ++ks) {
-                const uint32_t aoff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                const uint32_t boff = static_cast<uint32_t>(sp * C::NCB * C::CAP * 128 +
-                                                            (ks >> 2) * C::CAP * 128 + p0 * 128 +
-                                                            (ks & 3) * 32);
-                mma_ss_elect(tmem + wg * C::PIECE, smem_desc_sw128(qa + aoff, 16, 1024),
-                             smem_desc_sw128(sBa + boff, 16, 1024), idesc,
-                             (sp > 0 || ks > 0) ? 1u : 0u);
-              }
-            }
-            mma_commit_elect(&bars->mma_done[wg]);
+          const uint32_t pc = npiece - 1;  // this piece's number
+          if (p0 + C::PIECE < n_t) {
+            if (ok && warp == wg * 4) issue(p0 + C::PIECE);
+            ++npiece;
           }
-          const bool w = ok && mbar_wait_bounded(&bars->mma_done[wg], mphase, abort_flag,
-                                                 status, kDevTimeoutAttn, TO);
-          mphase ^= 1;
+          const bool w = ok && mbar_wait_bounded(&bars->mma_done[wg][pc & 1], (pc >> 1) & 1,
+                                                 abort_flag, status, kDevTimeoutAttn, TO);
           // the Q buffer is free once the tile's last product is done: fetch the next one
           const bool last_pass = (c0 + n >= i_t || ch == nchunks - 1) && p0 + C::PIECE >= n_t;
           if (row == 0 && w && last_pass) {
@@ -280,9 +294,10 @@ __global__ void __launch_bounds__(256, 1)
           }
           if (__all_sync(0xffffffffu, w)) {
             tc_fence_after();
+            const uint32_t tb = t_s + (pc & 1) * C::PIECE;
             for (int cc = 0; cc < np; cc += 32) {
               uint32_t sr[32];
-              tmem_ld32(t_s + cc, sr);
+              tmem_ld32(tb + cc, sr);
               tmem_wait_ld();
 #pragma unroll
               for (int x = 0; x < 32; ++x) reg_fence(sr[x]);
@@ -290,24 +305,27 @@ __global__ void __launch_bounds__(256, 1)
               const float thr0 = vals[KCAP - 1];
               uint32_t mask = 0;
 #pragma unroll
-              for (int x = 0; x < 32; ++x) {
-                stage[x * 128 + row] = __uint_as_float(sr[x]);
+              for (int x = 0; x < 32; ++x)
                 if (cc + x < np && __uint_as_float(sr[x]) > thr0) mask |= 1u << x;
-              }
-              const int jb = c0 + p0 + cc;
-              while (__any_sync(0xffffffffu, mask != 0)) {
-                if (mask) {
-                  const int x = __ffs(mask) - 1;
-                  mask &= mask - 1;
-                  const float sc = stage[x * 128 + row];
-                  if (sc > vals[KCAP - 1]) insert_top<KCAP>(vals, ids, sc, jb + x);
+              if (__any_sync(0xffffffffu, mask != 0)) {
+                // stage this thread's scores so that a candidate can be picked by its column
+#pragma unroll
+                for (int x = 0; x < 32; ++x) stage[x * 128 + row] = __uint_as_float(sr[x]);
+                const int jb = c0 + p0 + cc;
+                while (__any_sync(0xffffffffu, mask != 0)) {
+                  if (mask) {
+                    const int x = __ffs(mask) - 1;
+                    mask &= mask - 1;
+                    const float sc = stage[x * 128 + row];
+                    if (sc > vals[KCAP - 1]) insert_top<KCAP>(vals, ids, sc, jb + x);
+                  }
                 }
+                __syncwarp();
               }
-              __syncwarp();
             }
             tc_fence_before();
           }
-          // every thread of the warpgroup has read the scores before the next pass overwrites them
+          // every thread of the warpgroup has read this buffer before piece p + 2 overwrites it
           ok = named_bar_and(1 + wg, 128, w);
         }
       }
