@@ -198,10 +198,10 @@ struct D64Cfg {
   static constexpr int HALF_BYTES = kTile * D * 2;  // 16 KB: one 128 x 64 bf16 tile
   static constexpr int Q_BYTES = 2 * HALF_BYTES;    // one 256-row item
   static constexpr int QB = 4;                      // Q buffers (items gathered ahead)
-  static constexpr int NST = 2;                     // K and V ring depth
+  static constexpr int NK = 2, NV = 3;              // K and V ring depths (V is freed later)
   static constexpr int OFF_K = QB * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NST * HALF_BYTES;
-  static constexpr int OFF_BARS = OFF_V + NST * HALF_BYTES;
+  static constexpr int OFF_V = OFF_K + NK * HALF_BYTES;
+  static constexpr int OFF_BARS = OFF_V + NV * HALF_BYTES;
   static constexpr int SMEM_BYTES = OFF_BARS + 8192;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t REGS_CTRL = 72, REGS_SOFTMAX = 216;  // 128*72 + 256*216 = 384*168
@@ -216,13 +216,12 @@ static_assert(D64Cfg::SMEM_BYTES <= 232448, "shared memory budget of one CTA");
 
 struct D64Bars {
   uint64_t q_full[D64Cfg::QB], q_empty[D64Cfg::QB];
-  uint64_t k_full[D64Cfg::NST], k_empty[D64Cfg::NST], v_full[D64Cfg::NST], v_empty[D64Cfg::NST];
+  uint64_t k_full[D64Cfg::NK], k_empty[D64Cfg::NK], v_full[D64Cfg::NV], v_empty[D64Cfg::NV];
   uint64_t s_full[2], p_full[2], o_full[2][2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
   ItemRing ring;
-  int q_row[kItemRows];  // gather scratch: query row (t * H + h) of each item row, -1 = none
   // per softmax thread: the previous item's output row (-1 = none), 1 / l and log-sum-exp
   int ep_row[kItemRows];
   float ep_inv[kItemRows], ep_lse[kItemRows];
@@ -252,9 +251,11 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->q_full[x], 32);
       mbar_init(&bars->q_empty[x], 1);
     }
-    for (int x = 0; x < C::NST; ++x) {
+    for (int x = 0; x < C::NK; ++x) {
       mbar_init(&bars->k_full[x], 1);
       mbar_init(&bars->k_empty[x], 1);
+    }
+    for (int x = 0; x < C::NV; ++x) {
       mbar_init(&bars->v_full[x], 1);
       mbar_init(&bars->v_empty[x], 1);
     }
@@ -303,20 +304,19 @@ __global__ void __launch_bounds__(384, 1)
         ok = __all_sync(0xffffffffu, pop(lt, it));
         if (!ok || it.kind < 0) break;
         for (int j = 0; j < it.nsub; ++j, ++J) {
-          const int st = J % C::NST;
-          const uint32_t ph = (J / C::NST) & 1;
+          const int sk = J % C::NK, sv = J % C::NV;
           const int tok = it.key0 + j * kTile;
-          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->k_empty[st], ph ^ 1, abort_flag,
-                                                         err, kDevTimeoutAttn, TO));
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->k_empty[sk], ((J / C::NK) & 1) ^ 1,
+                                                         abort_flag, err, kDevTimeoutAttn, TO));
           if (!ok) break;
-          mbar_arrive_expect_tx_elect(&bars->k_full[st], C::HALF_BYTES);
-          tma_load_3d_elect(sK + st * C::HALF_BYTES, &map_k, &bars->k_full[st], 0, it.g, tok);
+          mbar_arrive_expect_tx_elect(&bars->k_full[sk], C::HALF_BYTES);
+          tma_load_3d_elect(sK + sk * C::HALF_BYTES, &map_k, &bars->k_full[sk], 0, it.g, tok);
           ++issued_k;
-          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->v_empty[st], ph ^ 1, abort_flag,
-                                                         err, kDevTimeoutAttn, TO));
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->v_empty[sv], ((J / C::NV) & 1) ^ 1,
+                                                         abort_flag, err, kDevTimeoutAttn, TO));
           if (!ok) break;
-          mbar_arrive_expect_tx_elect(&bars->v_full[st], C::HALF_BYTES);
-          tma_load_3d_elect(sV + st * C::HALF_BYTES, &map_v, &bars->v_full[st], 0, it.g, tok);
+          mbar_arrive_expect_tx_elect(&bars->v_full[sv], C::HALF_BYTES);
+          tma_load_3d_elect(sV + sv * C::HALF_BYTES, &map_v, &bars->v_full[sv], 0, it.g, tok);
           ++issued_v;
         }
         if (!ok) break;
@@ -324,17 +324,15 @@ __global__ void __launch_bounds__(384, 1)
       if (!ok) {
         // after an abort, let the loads still in flight land before the CTA exits (bounded)
         volatile int no_abort = 0;
-        for (uint32_t x = 0; x < static_cast<uint32_t>(C::NST); ++x) {
-          if (issued_k > x) {
-            const uint32_t Jx = issued_k - 1 - x;
-            mbar_wait_bounded(&bars->k_full[Jx % C::NST], (Jx / C::NST) & 1, &no_abort, nullptr,
-                              0, TO / 4);
-          }
-          if (issued_v > x) {
-            const uint32_t Jx = issued_v - 1 - x;
-            mbar_wait_bounded(&bars->v_full[Jx % C::NST], (Jx / C::NST) & 1, &no_abort, nullptr,
-                              0, TO / 4);
-          }
+        for (uint32_t x = 0; x < static_cast<uint32_t>(C::NK) && x < issued_k; ++x) {
+          const uint32_t Jx = issued_k - 1 - x;
+          mbar_wait_bounded(&bars->k_full[Jx % C::NK], (Jx / C::NK) & 1, &no_abort, nullptr, 0,
+                            TO / 4);
+        }
+        for (uint32_t x = 0; x < static_cast<uint32_t>(C::NV) && x < issued_v; ++x) {
+          const uint32_t Jx = issued_v - 1 - x;
+          mbar_wait_bounded(&bars->v_full[Jx % C::NV], (Jx / C::NV) & 1, &no_abort, nullptr, 0,
+                            TO / 4);
         }
       }
     } else if (warp == 1) {
@@ -350,34 +348,34 @@ __global__ void __launch_bounds__(384, 1)
         return __all_sync(0xffffffffu,
                           mbar_wait_bounded(bar, parity, abort_flag, err, kDevTimeoutAttn, TO));
       };
-      auto issue_s = [&](int half, uint32_t qb, int st) {
+      auto issue_s = [&](int half, uint32_t qb, int sk) {
         const uint64_t ad = smem_desc_sw128(sQa + qb * C::Q_BYTES + half * C::HALF_BYTES, 16, 1024);
-        const uint64_t bd = smem_desc_sw128(sKa + st * C::HALF_BYTES, 16, 1024);
+        const uint64_t bd = smem_desc_sw128(sKa + sk * C::HALF_BYTES, 16, 1024);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
           mma_ss_elect(tmem + C::tm_s(half), desc_advance(ad, ks * 32), desc_advance(bd, ks * 32),
                        IDESC_QK, ks > 0 ? 1u : 0u);
         mma_commit_elect(&bars->s_full[half]);
       };
-      // O_x += P_x V_st for the half's sub-tile number c of its item number item
-      auto issue_pv = [&](int half, int st, uint32_t c, uint32_t item, bool first, bool last,
+      // O_x += P_x V_sv for the half's sub-tile number c of its item number item
+      auto issue_pv = [&](int half, int sv, uint32_t c, uint32_t item, bool first, bool last,
                           bool free_v) -> bool {
         if (!wait(&bars->p_full[half], c & 1)) return false;
         tc_fence_after();
         const uint32_t t_o = tmem + C::tm_o(half, item & 1);
         const uint32_t t_p = tmem + C::tm_s(half);
-        const uint64_t bd = smem_desc_sw128(sVa + st * C::HALF_BYTES, 16384, 1024);
+        const uint64_t bd = smem_desc_sw128(sVa + sv * C::HALF_BYTES, 16384, 1024);
 #pragma unroll
         for (int ks = 0; ks < kTile / 16; ++ks)
           mma_ts_elect(t_o, t_p + ks * 8, desc_advance(bd, ks * 2048), IDESC_PV,
                        (first && ks == 0) ? 0u : 1u);
-        if (free_v) mma_commit_elect(&bars->v_empty[st]);
+        if (free_v) mma_commit_elect(&bars->v_empty[sv]);
         if (last) mma_commit_elect(&bars->o_full[half][item & 1]);
         return true;
       };
       // PV of half B is issued one step late, after the next S of half A (ping-pong)
       bool pend = false, pend_first = false, pend_last = false;
-      int pend_st = 0;
+      int pend_sv = 0;
       uint32_t pend_c = 0, pend_item = 0;
       for (uint32_t lt = 0;; ++lt) {
         Item it;
@@ -389,27 +387,27 @@ __global__ void __launch_bounds__(384, 1)
         if (!ok) break;
         tc_fence_after();
         for (int j = 0; j < it.nsub; ++j, ++J) {
-          const int st = J % C::NST;
-          ok = wait(&bars->k_full[st], (J / C::NST) & 1);
+          const int sk = J % C::NK, sv = J % C::NV;
+          ok = wait(&bars->k_full[sk], (J / C::NK) & 1);
           if (!ok) break;
           tc_fence_after();
-          issue_s(0, qb, st);
+          issue_s(0, qb, sk);
           if (pend) {
             pend = false;
-            ok = issue_pv(1, pend_st, pend_c, pend_item, pend_first, pend_last, true);
+            ok = issue_pv(1, pend_sv, pend_c, pend_item, pend_first, pend_last, true);
             if (!ok) break;
           }
-          if (hasB) issue_s(1, qb, st);
-          mma_commit_elect(&bars->k_empty[st]);
+          if (hasB) issue_s(1, qb, sk);
+          mma_commit_elect(&bars->k_empty[sk]);
           if (j == it.nsub - 1) mma_commit_elect(&bars->q_empty[qb]);
-          ok = wait(&bars->v_full[st], (J / C::NST) & 1);
+          ok = wait(&bars->v_full[sv], (J / C::NV) & 1);
           if (!ok) break;
-          ok = issue_pv(0, st, cs[0], ci[0], j == 0, j == it.nsub - 1, !hasB);
+          ok = issue_pv(0, sv, cs[0], ci[0], j == 0, j == it.nsub - 1, !hasB);
           if (!ok) break;
           ++cs[0];
           if (hasB) {
             pend = true;
-            pend_st = st;
+            pend_sv = sv;
             pend_c = cs[1]++;
             pend_item = ci[1];
             pend_first = (j == 0);
@@ -420,7 +418,7 @@ __global__ void __launch_bounds__(384, 1)
         ++ci[0];
         if (hasB) ++ci[1];
       }
-      if (ok && pend) ok = issue_pv(1, pend_st, pend_c, pend_item, pend_first, pend_last, true);
+      if (ok && pend) ok = issue_pv(1, pend_sv, pend_c, pend_item, pend_first, pend_last, true);
       if (!ok) {
         // after an abort, wait (bounded) until the MMAs already issued have finished with TMEM
         volatile int no_abort = 0;
@@ -430,55 +428,69 @@ __global__ void __launch_bounds__(384, 1)
     } else if (warp == 2) {
       // ------------------------------------------------------------------ Q row gather
       // Item rows are spread 4 per warp instruction (8 lanes x 16 bytes = one 128-byte row), so
-      // every copy instruction moves four whole rows.
+      // every copy instruction moves four whole rows. The routing entries of the next item are
+      // read (coalesced, one per lane and 32-row group) while this item's rows are copied, and a
+      // row's query index reaches the 8 lanes that copy it by a shuffle.
       const uint32_t sQa = smem_u32(sQ);
-      int* q_row = bars->q_row;
+      const int c = lane & 7, r0 = lane >> 3;
       bool ok = true, pending = false;
       uint32_t prev_qb = 0;
-      for (uint32_t lt = 0;; ++lt) {
+      auto fetch = [&](const Item& it, int (&e)[kItemRows / 32]) {
+#pragma unroll
+        for (int u = 0; u < kItemRows / 32; ++u) {
+          const int m = lane + 32 * u;
+          e[u] = (it.kind == 1 && m < it.rows) ? __ldg(a.entries + it.start + m) : 0;
+        }
+      };
+      Item cur;
+      int ecur[kItemRows / 32];
+      ok = __all_sync(0xffffffffu, pop(0, cur));
+      if (ok) fetch(cur, ecur);
+      for (uint32_t lt = 0; ok && cur.kind >= 0; ++lt) {
         const uint32_t qb = lt % C::QB;
         const uint32_t par = ((lt / C::QB) & 1) ^ 1;
-        // publish the previous item first whenever the next one cannot start at once (keeps the
+        // publish the previous item first whenever the next step cannot start at once (keeps the
         // MMA fed, and no wait below ever holds back an item the other roles need)
-        if (pending && !__all_sync(0xffffffffu, ring_ready(ring, lt) &&
+        if (pending && !__all_sync(0xffffffffu, ring_ready(ring, lt + 1) &&
                                                     mbar_try_wait(&bars->q_empty[qb], par))) {
           cp_async_wait_group<0>();
           fence_proxy_async_smem();
           mbar_arrive(&bars->q_full[prev_qb]);
           pending = false;
         }
-        Item it;
-        ok = __all_sync(0xffffffffu, pop(lt, it));
-        if (!ok || it.kind < 0) break;
+        Item nxt;
+        ok = __all_sync(0xffffffffu, pop(lt + 1, nxt));
+        if (!ok) break;
+        int enxt[kItemRows / 32];
+        fetch(nxt, enxt);
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->q_empty[qb], par, abort_flag, err,
                                                        kDevTimeoutAttn, TO));
         if (!ok) break;
-        // query row of every item row; the routing entries are read with coalesced loads first
-        int ent[kItemRows / 32];
+        // query row (t * H + h) of item rows lane + 32 u, -1 = padding
+        int qrow[kItemRows / 32];
 #pragma unroll
         for (int u = 0; u < kItemRows / 32; ++u) {
           const int m = lane + 32 * u;
-          ent[u] = (it.kind == 1 && m < it.rows) ? __ldg(a.entries + it.start + m) : 0;
+          qrow[u] = -1;
+          if (m < cur.rows)
+            qrow[u] = (cur.kind == 1) ? a.T0 * a.H + ecur[u] / a.topk : (cur.qtok0 + m) * a.H + cur.h;
         }
-#pragma unroll
-        for (int u = 0; u < kItemRows / 32; ++u) {
-          const int m = lane + 32 * u;
-          int qr = -1;
-          if (m < it.rows)
-            qr = (it.kind == 1) ? a.T0 * a.H + ent[u] / a.topk : (it.qtok0 + m) * a.H + it.h;
-          q_row[m] = qr;
-        }
-        __syncwarp();
-        const int nrows = it.rows > kTile ? kItemRows : kTile;
         const uint32_t dst0 = sQa + qb * C::Q_BYTES;
-        const int c = lane & 7;
-        for (int m = lane >> 3; m < nrows; m += 4) {
-          const int qr = q_row[m];
+        // row m = 4 i + r0, chunk c; its query row sits in lane m % 32, register m / 32
+        auto copy = [&](int i) {
+          const int m = 4 * i + r0;
+          const int qr = __shfl_sync(0xffffffffu, qrow[i / 8], (4 * i) % 32 + r0);
           const __nv_bfloat16* src = (qr >= 0) ? a.q + static_cast<size_t>(qr) * D + c * 8 : a.q;
-          const uint32_t dst = dst0 + (m >> 7) * C::HALF_BYTES + sw128_offset(m & 127, c * 8);
-          cp_async_16(dst, src, qr >= 0 ? 16u : 0u);
+          cp_async_16(dst0 + (m >> 7) * C::HALF_BYTES + sw128_offset(m & 127, c * 8), src,
+                      qr >= 0 ? 16u : 0u);
+        };
+        if (cur.rows > kTile) {
+#pragma unroll
+          for (int i = 0; i < kItemRows / 4; ++i) copy(i);
+        } else {
+#pragma unroll
+          for (int i = 0; i < kTile / 4; ++i) copy(i);
         }
-        __syncwarp();
         cp_async_commit();
         if (pending) {
           cp_async_wait_group<1>();
@@ -487,6 +499,9 @@ __global__ void __launch_bounds__(384, 1)
         }
         pending = true;
         prev_qb = qb;
+        cur = nxt;
+#pragma unroll
+        for (int u = 0; u < kItemRows / 32; ++u) ecur[u] = enxt[u];
       }
       cp_async_wait_all();
       if (ok && pending) {
