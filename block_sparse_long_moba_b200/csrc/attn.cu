@@ -230,7 +230,8 @@ static_assert(sizeof(D64Bars) <= 8192, "barrier block");
 
 __global__ void __launch_bounds__(384, 1)
     attn_kernel_d64(const __grid_constant__ CUtensorMap map_k,
-                    const __grid_constant__ CUtensorMap map_v, const AttnArgs a) {
+                    const __grid_constant__ CUtensorMap map_v,
+                    const __grid_constant__ CUtensorMap map_q, const AttnArgs a) {
   using C = D64Cfg;
   constexpr int D = C::D;
   extern __shared__ __align__(1024) uint8_t smem64[];
@@ -248,7 +249,7 @@ __global__ void __launch_bounds__(384, 1)
   }
   if (tid == 0) {
     for (int x = 0; x < C::QB; ++x) {
-      mbar_init(&bars->q_full[x], 32);
+      mbar_init(&bars->q_full[x], 1);
       mbar_init(&bars->q_empty[x], 1);
     }
     for (int x = 0; x < C::NK; ++x) {
@@ -280,6 +281,7 @@ __global__ void __launch_bounds__(384, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&map_k);
     prefetch_tensormap(&map_v);
+    prefetch_tensormap(&map_q);
   }
   tc_fence_before();
   __syncthreads();
@@ -427,86 +429,63 @@ __global__ void __launch_bounds__(384, 1)
       }
     } else if (warp == 2) {
       // ------------------------------------------------------------------ Q row gather
-      // Item rows are spread 4 per warp instruction (8 lanes x 16 bytes = one 128-byte row), so
-      // every copy instruction moves four whole rows. The routing entries of the next item are
-      // read (coalesced, one per lane and 32-row group) while this item's rows are copied, and a
-      // row's query index reaches the 8 lanes that copy it by a shuffle.
-      const uint32_t sQa = smem_u32(sQ);
-      const int c = lane & 7, r0 = lane >> 3;
-      bool ok = true, pending = false;
-      uint32_t prev_qb = 0;
-      auto fetch = [&](const Item& it, int (&e)[kItemRows / 32]) {
+      // On the TMA unit: each lane gathers rows 4 lane .. 4 lane + 3 of each 128-row half with one
+      // tile::gather4 copy (four 128-byte rows, swizzled by the TMA unit into the layout the MMA
+      // reads); lane 0 posts the item's byte count on q_full first, so the warp never waits for
+      // the data. The routing entries of the next item are read while this one is in flight.
+      bool ok = true;
+      uint32_t issued = 0;
+      auto fetch = [&](const Item& it, int (&e)[8]) {
 #pragma unroll
-        for (int u = 0; u < kItemRows / 32; ++u) {
-          const int m = lane + 32 * u;
-          e[u] = (it.kind == 1 && m < it.rows) ? __ldg(a.entries + it.start + m) : 0;
+        for (int x = 0; x < 8; ++x) {
+          const int m = (x >> 2) * kTile + 4 * lane + (x & 3);
+          e[x] = (it.kind == 1 && m < it.rows) ? __ldg(a.entries + it.start + m) : 0;
         }
       };
       Item cur;
-      int ecur[kItemRows / 32];
+      int ecur[8];
       ok = __all_sync(0xffffffffu, pop(0, cur));
       if (ok) fetch(cur, ecur);
       for (uint32_t lt = 0; ok && cur.kind >= 0; ++lt) {
         const uint32_t qb = lt % C::QB;
-        const uint32_t par = ((lt / C::QB) & 1) ^ 1;
-        // publish the previous item first whenever the next step cannot start at once (keeps the
-        // MMA fed, and no wait below ever holds back an item the other roles need)
-        if (pending && !__all_sync(0xffffffffu, ring_ready(ring, lt + 1) &&
-                                                    mbar_try_wait(&bars->q_empty[qb], par))) {
-          cp_async_wait_group<0>();
-          fence_proxy_async_smem();
-          mbar_arrive(&bars->q_full[prev_qb]);
-          pending = false;
-        }
         Item nxt;
         ok = __all_sync(0xffffffffu, pop(lt + 1, nxt));
         if (!ok) break;
-        int enxt[kItemRows / 32];
+        int enxt[8];
         fetch(nxt, enxt);
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->q_empty[qb], par, abort_flag, err,
-                                                       kDevTimeoutAttn, TO));
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->q_empty[qb], ((lt / C::QB) & 1) ^ 1,
+                                                       abort_flag, err, kDevTimeoutAttn, TO));
         if (!ok) break;
-        // query row (t * H + h) of item rows lane + 32 u, -1 = padding
-        int qrow[kItemRows / 32];
+        const bool hasB = cur.rows > kTile;
+        // query row (t * H + h) of item row m; padding rows repeat a valid row (their results are
+        // never written)
+        int y[8];
 #pragma unroll
-        for (int u = 0; u < kItemRows / 32; ++u) {
-          const int m = lane + 32 * u;
-          qrow[u] = -1;
-          if (m < cur.rows)
-            qrow[u] = (cur.kind == 1) ? a.T0 * a.H + ecur[u] / a.topk : (cur.qtok0 + m) * a.H + cur.h;
+        for (int x = 0; x < 8; ++x) {
+          const int m = (x >> 2) * kTile + 4 * lane + (x & 3);
+          y[x] = (cur.kind == 1) ? a.T0 * a.H + ecur[x] / a.topk
+                                 : (cur.qtok0 + (m < cur.rows ? m : 0)) * a.H + cur.h;
         }
-        const uint32_t dst0 = sQa + qb * C::Q_BYTES;
-        // row m = 4 i + r0, chunk c; its query row sits in lane m % 32, register m / 32
-        auto copy = [&](int i) {
-          const int m = 4 * i + r0;
-          const int qr = __shfl_sync(0xffffffffu, qrow[i / 8], (4 * i) % 32 + r0);
-          const __nv_bfloat16* src = (qr >= 0) ? a.q + static_cast<size_t>(qr) * D + c * 8 : a.q;
-          cp_async_16(dst0 + (m >> 7) * C::HALF_BYTES + sw128_offset(m & 127, c * 8), src,
-                      qr >= 0 ? 16u : 0u);
-        };
-        if (cur.rows > kTile) {
-#pragma unroll
-          for (int i = 0; i < kItemRows / 4; ++i) copy(i);
-        } else {
-#pragma unroll
-          for (int i = 0; i < kTile / 4; ++i) copy(i);
-        }
-        cp_async_commit();
-        if (pending) {
-          cp_async_wait_group<1>();
-          fence_proxy_async_smem();
-          mbar_arrive(&bars->q_full[prev_qb]);
-        }
-        pending = true;
-        prev_qb = qb;
+        if (lane == 0)
+          mbar_arrive_expect_tx(&bars->q_full[qb], (hasB ? 2 : 1) * C::HALF_BYTES);
+        __syncwarp();
+        uint8_t* dst = sQ + qb * C::Q_BYTES + lane * 512;
+        tma_gather4(dst, &map_q, &bars->q_full[qb], 0, y[0], y[1], y[2], y[3]);
+        if (hasB)
+          tma_gather4(dst + C::HALF_BYTES, &map_q, &bars->q_full[qb], 0, y[4], y[5], y[6], y[7]);
+        ++issued;
         cur = nxt;
 #pragma unroll
-        for (int u = 0; u < kItemRows / 32; ++u) ecur[u] = enxt[u];
+        for (int x = 0; x < 8; ++x) ecur[x] = enxt[x];
       }
-      cp_async_wait_all();
-      if (ok && pending) {
-        fence_proxy_async_smem();
-        mbar_arrive(&bars->q_full[prev_qb]);
+      if (!ok) {
+        // after an abort, let the gathers still in flight land before the CTA exits (bounded)
+        volatile int no_abort = 0;
+        for (uint32_t x = 0; x < static_cast<uint32_t>(C::QB) && x < issued; ++x) {
+          const uint32_t l = issued - 1 - x;
+          mbar_wait_bounded(&bars->q_full[l % C::QB], (l / C::QB) & 1, &no_abort, nullptr, 0,
+                            TO / 4);
+        }
       }
     } else {
       // ------------------------------------------------------------------ item scheduler
@@ -1169,9 +1148,25 @@ static bool make_kv_map(CUtensorMap* map, const void* base, int T, int G, int D)
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [T * H, D] bf16 query rows -> 2-D map (D, T * H), box (64, 1): one row per box, as the row
+// gather (tile::gather4) requires; 128-byte swizzle.
+static bool make_q_rows_map(CUtensorMap* map, const void* base, long long rows, int D) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t es[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream) {
-  CUtensorMap mk, mv;
+  CUtensorMap mk, mv, mq;
   if (!make_kv_map(&mk, L.k, L.T, L.G, L.d) || !make_kv_map(&mv, L.v, L.T, L.G, L.d))
+    return cudaErrorInvalidValue;
+  if (L.d == 64 && !make_q_rows_map(&mq, L.q, static_cast<long long>(L.T) * L.H, L.d))
     return cudaErrorInvalidValue;
   AttnArgs a;
   a.q = static_cast<const __nv_bfloat16*>(L.q);
@@ -1209,7 +1204,7 @@ cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream) {
     const int smem = D64Cfg::SMEM_BYTES;
     cudaError_t e = cudaFuncSetAttribute(attn_kernel_d64, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_kernel_d64<<<grid, 384, smem, stream>>>(mk, mv, a);
+    attn_kernel_d64<<<grid, 384, smem, stream>>>(mk, mv, mq, a);
   } else {
     const int smem = PvtCfg::SMEM_BYTES;
     cudaError_t e = cudaFuncSetAttribute(attn_kernel_pvt, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -59,26 +59,86 @@ __device__ __forceinline__ uint32_t c_offset(int s, int row, int col) {
          sw128_offset(row, col & 63);
 }
 
-// Inserts (s, j) into the list sorted best first; requires s > vals[KCAP - 1]. An entry equal to s
-// stays ahead of it. gt[] is monotone (the list is sorted), so position x takes the entry above it
-// when s beats that one, s when s beats only the entry at x, and keeps its entry otherwise.
-template <int KCAP>
-__device__ __forceinline__ void insert_top(float (&vals)[KCAP], int (&ids)[KCAP], float s, int j) {
-  bool gt[KCAP];
-#pragma unroll
-  for (int x = 0; x < KCAP; ++x) gt[x] = s > vals[x];
-#pragma unroll
-  for (int x = KCAP - 1; x > 0; --x) {
-    vals[x] = gt[x - 1] ? vals[x - 1] : (gt[x] ? s : vals[x]);
-    ids[x] = gt[x - 1] ? ids[x - 1] : (gt[x] ? j : ids[x]);
-  }
-  vals[0] = gt[0] ? s : vals[0];
-  ids[0] = gt[0] ? j : ids[0];
+// Order-preserving map of fp32 to uint32 (a larger float gives a larger unsigned) and back.
+__device__ __forceinline__ uint32_t f2ord(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
+__device__ __forceinline__ float ord2f(uint32_t o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
+// Running top list of one row, best first. The first KCAP - ksel places hold sentinels that no
+// score displaces, so the last place is always the ksel-th best so far: the exact threshold.
+template <int KCAP, bool PACK>
+struct TopList;
+
+// Scores and block ids kept apart; equal scores keep the earlier (lower) block.
+template <int KCAP>
+struct TopList<KCAP, false> {
+  float v[KCAP];
+  int id[KCAP];
+  __device__ __forceinline__ void init(int ksel) {
+#pragma unroll
+    for (int x = 0; x < KCAP; ++x) {
+      v[x] = (x < KCAP - ksel) ? INFINITY : -INFINITY;
+      id[x] = 0x7fffffff;
+    }
+  }
+  // columns worth a closer look: s > thr with thr read once per 32 columns
+  __device__ __forceinline__ float thr() const { return v[KCAP - 1]; }
+  __device__ __forceinline__ static bool cand(float s, float t) { return s > t; }
+  // Inserts (s, j) if it beats the last place. gt[] is monotone (the list is sorted), so position
+  // x takes the entry above it when s beats that one, s when s beats only the entry at x, and
+  // keeps its entry otherwise: every position is computed independently.
+  __device__ __forceinline__ void offer(float s, int j) {
+    if (!(s > v[KCAP - 1])) return;
+    bool gt[KCAP];
+#pragma unroll
+    for (int x = 0; x < KCAP; ++x) gt[x] = s > v[x];
+#pragma unroll
+    for (int x = KCAP - 1; x > 0; --x) {
+      v[x] = gt[x - 1] ? v[x - 1] : (gt[x] ? s : v[x]);
+      id[x] = gt[x - 1] ? id[x - 1] : (gt[x] ? j : id[x]);
+    }
+    v[0] = gt[0] ? s : v[0];
+    id[0] = gt[0] ? j : id[0];
+  }
+  __device__ __forceinline__ int block(int x) const { return id[x]; }
+};
+
+// One 32-bit key per entry, for sequences of at most 256 blocks: the order-preserving image of
+// the score with its low 8 bits replaced by 255 - block, so keys are distinct, a larger key is a
+// better score, and equal truncated scores rank the lower block first. The truncation changes an
+// order only between scores within 2^-15 of each other (relative), inside the near-tie band of the
+// routing rule. An insertion is then KCAP integer max and KCAP - 1 min operations.
+template <int KCAP>
+struct TopList<KCAP, true> {
+  uint32_t k[KCAP];
+  __device__ __forceinline__ void init(int ksel) {
+#pragma unroll
+    for (int x = 0; x < KCAP; ++x) k[x] = (x < KCAP - ksel) ? 0xffffffffu : 0u;
+  }
+  // a key can only beat the last place if its score is at least this
+  __device__ __forceinline__ float thr() const {
+    return k[KCAP - 1] == 0u ? -INFINITY : ord2f(k[KCAP - 1] & ~0xffu);
+  }
+  __device__ __forceinline__ static bool cand(float s, float t) { return s >= t; }
+  __device__ __forceinline__ void offer(float s, int j) {
+    const uint32_t key = (f2ord(s) & ~0xffu) | static_cast<uint32_t>(255 - j);
+    if (key <= k[KCAP - 1]) return;
+#pragma unroll
+    for (int x = KCAP - 1; x > 0; --x) k[x] = max(k[x], min(k[x - 1], key));
+    k[0] = max(k[0], key);
+  }
+  __device__ __forceinline__ int block(int x) const {
+    return k[x] == 0xffffffffu ? 0x7fffffff : 255 - static_cast<int>(k[x] & 0xffu);
+  }
+};
 
 }  // namespace
 
-template <int D, int KCAP>
+template <int D, int KCAP, bool PACK>
 __global__ void __launch_bounds__(256, 1)
     gate_tc_kernel(const __grid_constant__ CUtensorMap map_q, const float* __restrict__ cents,
                    const int32_t* __restrict__ cu, int nseq, int max_nb, int T, int H, int G,
@@ -198,13 +258,8 @@ __global__ void __launch_bounds__(256, 1)
         else
           for (int x = 0; x < topk; ++x) out[x] = (x <= i_t) ? x : -1;
       }
-      float vals[KCAP];
-      int ids[KCAP];
-#pragma unroll
-      for (int x = 0; x < KCAP; ++x) {
-        vals[x] = -INFINITY;
-        ids[x] = 0x7fffffff;
-      }
+      TopList<KCAP, PACK> top;
+      top.init(ksel);
       bool q_ready = false;
       for (int ch = 0; ch < nchunks; ++ch) {
         const int c0 = ch * C::CAP;
@@ -302,11 +357,11 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
               for (int x = 0; x < 32; ++x) reg_fence(sr[x]);
               // candidates: columns that beat this row's current threshold
-              const float thr0 = vals[KCAP - 1];
+              const float thr0 = top.thr();
               uint32_t mask = 0;
 #pragma unroll
               for (int x = 0; x < 32; ++x)
-                if (cc + x < np && __uint_as_float(sr[x]) > thr0) mask |= 1u << x;
+                if (cc + x < np && top.cand(__uint_as_float(sr[x]), thr0)) mask |= 1u << x;
               if (__any_sync(0xffffffffu, mask != 0)) {
                 // stage this thread's scores so that a candidate can be picked by its column
 #pragma unroll
@@ -316,8 +371,7 @@ __global__ void __launch_bounds__(256, 1)
                   if (mask) {
                     const int x = __ffs(mask) - 1;
                     mask &= mask - 1;
-                    const float sc = stage[x * 128 + row];
-                    if (sc > vals[KCAP - 1]) insert_top<KCAP>(vals, ids, sc, jb + x);
+                    top.offer(stage[x * 128 + row], jb + x);
                   }
                 }
                 __syncwarp();
@@ -330,18 +384,17 @@ __global__ void __launch_bounds__(256, 1)
         }
       }
       if (!scored || row >= rows || !ok) continue;
+      // the ksel real entries (sentinels map to INT_MAX), ascending
       int sel[KCAP];
 #pragma unroll
-      for (int x = 0; x < KCAP; ++x) sel[x] = (x < ksel) ? ids[x] : 0x7fffffff;
+      for (int x = 0; x < KCAP; ++x) sel[x] = top.block(x);
 #pragma unroll
       for (int a0 = 0; a0 < KCAP - 1; ++a0) {
 #pragma unroll
         for (int b0 = 0; b0 < KCAP - 1 - a0; ++b0) {
-          if (sel[b0] > sel[b0 + 1]) {
-            const int tmp = sel[b0];
-            sel[b0] = sel[b0 + 1];
-            sel[b0 + 1] = tmp;
-          }
+          const int lo_ = min(sel[b0], sel[b0 + 1]), hi_ = max(sel[b0], sel[b0 + 1]);
+          sel[b0] = lo_;
+          sel[b0 + 1] = hi_;
         }
       }
       int32_t* out = idx + (static_cast<size_t>(h) * T + t0 + row) * topk;
@@ -389,17 +442,29 @@ bool make_q_map(CUtensorMap* map, const void* q, int T, int H, int D) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int D, int KCAP, bool PACK>
+cudaError_t launch_tp(const CUtensorMap& mq, const float* cents, const int32_t* cu, int nseq,
+                      int max_nb, int T, int H, int G, int B, int topk, int32_t* idx, int* status,
+                      int grid, cudaStream_t stream) {
+  const int smem = GateCfg<D>::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(gate_tc_kernel<D, KCAP, PACK>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  gate_tc_kernel<D, KCAP, PACK><<<grid, 256, smem, stream>>>(mq, cents, cu, nseq, max_nb, T, H,
+                                                             G, B, topk, idx, status);
+  return cudaGetLastError();
+}
+
+// Packed keys need every block id of a sequence to fit in 8 bits.
 template <int D, int KCAP>
 cudaError_t launch_t(const CUtensorMap& mq, const float* cents, const int32_t* cu, int nseq,
                      int max_nb, int T, int H, int G, int B, int topk, int32_t* idx, int* status,
                      int grid, cudaStream_t stream) {
-  const int smem = GateCfg<D>::SMEM_BYTES;
-  cudaError_t e = cudaFuncSetAttribute(gate_tc_kernel<D, KCAP>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  gate_tc_kernel<D, KCAP><<<grid, 256, smem, stream>>>(mq, cents, cu, nseq, max_nb, T, H, G, B,
-                                                       topk, idx, status);
-  return cudaGetLastError();
+  if (max_nb <= 256)
+    return launch_tp<D, KCAP, true>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status,
+                                    grid, stream);
+  return launch_tp<D, KCAP, false>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status,
+                                   grid, stream);
 }
 
 template <int D>
