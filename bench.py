@@ -207,6 +207,36 @@ def oracle_sample_rate(w: wl.Workload, q, k, v, target_s: float = 15.0, seed: in
                       f"({t_cent:.1f} s, charged pro rata {done_tok}/{T})"}
 
 
+# ---------------------------------------------------------------------------------- traffic
+ATTN_SOURCES = ("attn.cu", "sm100.cuh", "common.cuh")
+
+
+def attention_source_hash() -> str:
+    """sha256 over the attention kernel's source files, in a fixed order."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for name in ATTN_SOURCES:
+        with open(os.path.join(ROOT, "block_sparse_long_moba_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def attention_traffic(workload: str):
+    """DRAM bytes (read + write) of one attention launch on `workload`, from the committed ncu
+    summary profiles/attention_<workload>_traffic.json, or None when there is none or it was taken
+    on other kernel sources than the ones being timed."""
+    path = os.path.join(ROOT, "profiles", f"attention_{workload}_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        if rec.get("kernel_sources_sha256") != attention_source_hash():
+            return None
+        return float(rec["bytes_per_launch"])
+    except Exception:
+        return None
+
+
 # ------------------------------------------------------------------------------- distributed
 def dist_setup(n_gpus: int):
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -361,14 +391,7 @@ def run_ours(args):
             kern[name] = ent
         if "gate" in kern:
             kern["gate"]["gate_tflops_fp32"] = gate_flops(w) / (kern["gate"]["ms_per_launch"] / 1e3) / 1e12
-        traffic = None
-        tpath = os.path.join(ROOT, "profiles", f"attention_{w.name}_traffic.json")
-        if os.path.exists(tpath):
-            try:
-                with open(tpath) as f:
-                    traffic = json.load(f).get("bytes_per_launch")
-            except Exception:
-                traffic = None
+        traffic = attention_traffic(w.name)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,

@@ -74,3 +74,20 @@ def test_max_over_ranks_two_gloo_ranks():
         p.join(120)
         assert p.exitcode == 0
     assert out[0] == 15.0 and out[1] == 15.0
+
+
+def test_attention_traffic_only_for_the_sources_it_was_taken_on(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    csrc = tmp_path / "block_sparse_long_moba_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for name in bench.ATTN_SOURCES:
+        (csrc / name).write_text("// " + name)
+    (tmp_path / "profiles").mkdir()
+    rec = tmp_path / "profiles" / "attention_w_traffic.json"
+    assert bench.attention_traffic("w") is None  # no record
+    import json
+    rec.write_text(json.dumps({"bytes_per_launch": 123.0,
+                               "kernel_sources_sha256": bench.attention_source_hash()}))
+    assert bench.attention_traffic("w") == 123.0
+    (csrc / "attn.cu").write_text("// changed")  # the kernel changed since the capture
+    assert bench.attention_traffic("w") is None
