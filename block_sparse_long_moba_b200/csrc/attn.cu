@@ -36,9 +36,22 @@ namespace moba {
 // Column pairs (of every 8) whose exp2 runs on the FMA pipe instead of MUFU.EX2, balancing the two.
 constexpr int kPolyPairs = 0;
 #ifndef MOBA_POLY_PAIRS_PVT
-#define MOBA_POLY_PAIRS_PVT 0
+#define MOBA_POLY_PAIRS_PVT 1
 #endif
 constexpr int kPolyPairsPvt = MOBA_POLY_PAIRS_PVT;
+
+// Partial outputs are written once and read once by the merge: with MOBA_PART_STREAM they are
+// stored with the evict-first policy so that they do not push the gathered query rows out of L2.
+#ifndef MOBA_PART_STREAM
+#define MOBA_PART_STREAM 1
+#endif
+__device__ __forceinline__ void st_part(uint4* p, uint4 v) {
+#if MOBA_PART_STREAM
+  __stcs(p, v);
+#else
+  *p = v;
+#endif
+}
 
 struct AttnArgs {
   const __nv_bfloat16* q;  // [T, H, D]
@@ -525,11 +538,11 @@ __global__ void __launch_bounds__(384, 1)
         if (prev_valid) {
 #pragma unroll
           for (int x = 0; x < 4; ++x)
-            dst[c0 / 8 + x] = make_uint4(
+            st_part(dst + c0 / 8 + x, make_uint4(
                 pack_bf16x2(__uint_as_float(orr[8 * x + 0]) * inv, __uint_as_float(orr[8 * x + 1]) * inv),
                 pack_bf16x2(__uint_as_float(orr[8 * x + 2]) * inv, __uint_as_float(orr[8 * x + 3]) * inv),
                 pack_bf16x2(__uint_as_float(orr[8 * x + 4]) * inv, __uint_as_float(orr[8 * x + 5]) * inv),
-                pack_bf16x2(__uint_as_float(orr[8 * x + 6]) * inv, __uint_as_float(orr[8 * x + 7]) * inv));
+                pack_bf16x2(__uint_as_float(orr[8 * x + 6]) * inv, __uint_as_float(orr[8 * x + 7]) * inv)));
         }
       }
       tc_fence_before();
@@ -739,7 +752,8 @@ __device__ __forceinline__ uint32_t p_offset(uint32_t row, uint32_t col) {
 
 __global__ void __launch_bounds__(384, 1)
     attn_kernel_pvt(const __grid_constant__ CUtensorMap map_k,
-                    const __grid_constant__ CUtensorMap map_v, const AttnArgs a) {
+                    const __grid_constant__ CUtensorMap map_v,
+                    const __grid_constant__ CUtensorMap map_q, const AttnArgs a) {
   using C = PvtCfg;
   constexpr int D = C::D;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -758,7 +772,7 @@ __global__ void __launch_bounds__(384, 1)
     return;
   }
   if (tid == 0) {
-    mbar_init(&bars->q_full, 64);
+    mbar_init(&bars->q_full, 33);  // warp 2 lane 0 (TMA bytes) + the 32 lanes of warp 3
     mbar_init(&bars->q_empty, 1);
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->k_full[x], 1);
@@ -781,6 +795,7 @@ __global__ void __launch_bounds__(384, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&map_k);
     prefetch_tensormap(&map_v);
+    prefetch_tensormap(&map_q);
   }
   tc_fence_before();
   __syncthreads();
@@ -911,41 +926,68 @@ __global__ void __launch_bounds__(384, 1)
       }
     } else {
       // ------------------------------------------------------------------ Q row gather
-      const int gt = tid - 64;  // 0..63
-      constexpr int CPR = D / 8;
+      // Two warps, two copy engines in parallel. Warp 2 gathers half A (rows 0..127) on the TMA
+      // unit with tile::gather4 (four rows x one 64-column box per copy, two boxes per row; lane 0
+      // posts the bytes on q_full first). Warp 3 copies half B (rows 128..255) with 16-byte
+      // cp.async, two 256-byte rows per warp instruction, and arrives once its copies have landed.
+      // Each lane reads the routing entries of four consecutive rows (coalesced over the warp);
+      // warp 3 hands the query-row index of a row to the 16 lanes that copy it by shuffles.
+      const int half = warp - 2;  // 0: rows 0..127 (TMA), 1: rows 128..255 (cp.async)
       uint32_t lt = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
         const Item it = decode_item(a, w, n_routed);
         if (it.kind == 0) continue;
-        ok = mbar_wait_bounded(&bars->q_empty, (lt & 1) ^ 1, abort_flag, err, kDevTimeoutAttn, TO);
-        if (!ok) break;
-        const uint32_t dst0 = smem_u32(sQ);
-        for (int e = gt; e < kItemRows * CPR; e += 64) {
-          const int m = e / CPR, c = e % CPR;
-          const __nv_bfloat16* src = a.q;
-          uint32_t bytes = 0;
-          if (m < it.rows) {
-            int t, h;
-            if (it.kind == 1) {
-              const int pr = __ldg(a.entries + it.start + m);
-              t = a.T0 + pr / (a.H * a.topk);
-              h = (pr / a.topk) % a.H;
-            } else {
-              t = it.qtok0 + m;
-              h = it.h;
-            }
-            src = a.q + (static_cast<size_t>(t) * a.H + h) * D + c * 8;
-            bytes = 16;
-          }
-          const uint32_t dst = dst0 + (m >> 7) * C::HALF_BYTES + (c >> 3) * 16384 +
-                               sw128_offset(m & 127, (c & 7) * 8);
-          cp_async_16(dst, src, bytes);
+        int qr4[4];  // query rows (t * H + h) of item rows half * 128 + 4 lane + r, -1 = padding
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int m = half * kTile + 4 * lane + r;
+          qr4[r] = (it.kind == 1 && m < it.rows) ? __ldg(a.entries + it.start + m) : 0;
         }
-        cp_async_wait_all();
-        fence_proxy_async_smem();
-        mbar_arrive(&bars->q_full);
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->q_empty, (lt & 1) ^ 1, abort_flag,
+                                                       err, kDevTimeoutAttn, TO));
+        if (!ok) break;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int m = half * kTile + 4 * lane + r;
+          // half A padding repeats a valid row for the TMA (never written back); half B padding
+          // is zero-filled by cp.async
+          qr4[r] = (m >= it.rows && half == 1) ? -1
+                   : (it.kind == 1) ? (m < it.rows ? a.T0 * a.H + qr4[r] / a.topk : a.T0 * a.H)
+                                    : (it.qtok0 + (m < it.rows ? m : 0)) * a.H + it.h;
+        }
+        if (half == 0) {
+          if (lane == 0) mbar_arrive_expect_tx(&bars->q_full, C::HALF_BYTES);
+          __syncwarp();
+          uint8_t* dst = sQ + lane * 512;
+          tma_gather4(dst, &map_q, &bars->q_full, 0, qr4[0], qr4[1], qr4[2], qr4[3]);
+          tma_gather4(dst + 16384, &map_q, &bars->q_full, 64, qr4[0], qr4[1], qr4[2], qr4[3]);
+        } else {
+          const uint32_t dst0 = smem_u32(sQ) + C::HALF_BYTES;
+          const int c = lane & 15, r0 = lane >> 4;
+          // instruction i copies rows 2 i and 2 i + 1 of half B, held by lane i / 2 in its
+          // registers 2 (i % 2) and 2 (i % 2) + 1
+#pragma unroll 8
+          for (int i = 0; i < kTile / 2; ++i) {
+            const int va = __shfl_sync(0xffffffffu, qr4[2 * (i & 1)], i >> 1);
+            const int vb = __shfl_sync(0xffffffffu, qr4[2 * (i & 1) + 1], i >> 1);
+            const int qr = r0 ? vb : va;
+            const int m = 2 * i + r0;
+            const __nv_bfloat16* src = (qr >= 0) ? a.q + static_cast<size_t>(qr) * D + c * 8 : a.q;
+            cp_async_16(dst0 + (c >> 3) * 16384 + sw128_offset(m, (c & 7) * 8), src,
+                        qr >= 0 ? 16u : 0u);
+          }
+          cp_async_wait_all();
+          fence_proxy_async_smem();
+          mbar_arrive(&bars->q_full);
+        }
         ++lt;
+      }
+      if (half == 1) cp_async_wait_all();
+      if (!ok && half == 0 && lt > 0) {
+        // after an abort, let the gathers still in flight land before the CTA exits (bounded)
+        volatile int no_abort = 0;
+        mbar_wait_bounded(&bars->q_full, (lt - 1) & 1, &no_abort, nullptr, 0, TO / 4);
       }
     }
   } else {
@@ -996,16 +1038,22 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < 128; ++c)
             if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
         }
+        // row max with three-input max: 8 running maxima over 16 columns per step
         float mx8[8];
 #pragma unroll
-        for (int x = 0; x < 8; ++x) mx8[x] = __uint_as_float(sr[x]);
+        for (int x = 0; x < 8; ++x)
+          mx8[x] = fmax3(__uint_as_float(sr[x]), __uint_as_float(sr[8 + x]),
+                         __uint_as_float(sr[16 + x]));
 #pragma unroll
-        for (int c = 8; c < 128; c += 8) {
+        for (int c = 24; c < 120; c += 16) {
 #pragma unroll
-          for (int x = 0; x < 8; ++x) mx8[x] = fmaxf(mx8[x], __uint_as_float(sr[c + x]));
+          for (int x = 0; x < 8; ++x)
+            mx8[x] = fmax3(mx8[x], __uint_as_float(sr[c + x]), __uint_as_float(sr[c + 8 + x]));
         }
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+#pragma unroll
+        for (int x = 0; x < 8; ++x) mx8[x] = fmaxf(mx8[x], __uint_as_float(sr[120 + x]));
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7]));
         const float mxs = mx * sl2;
         const bool need = mxs > m_ref + 8.f;
         float alpha = 1.f;
@@ -1020,9 +1068,14 @@ __global__ void __launch_bounds__(384, 1)
         auto exp_pair = [&](int c) -> uint32_t {
           float t0, t1;
           fma2(t0, t1, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), sl2, sl2, neg, neg);
-          const bool poly = ((c >> 1) & 7) >= 8 - kPolyPairsPvt;
-          const float p0 = poly ? exp2_poly(t0) : ex2_approx(t0);
-          const float p1 = poly ? exp2_poly(t1) : ex2_approx(t1);
+          // kPolyPairsPvt of every 8 column pairs run on the FMA pipe, the rest on MUFU.EX2
+          float p0, p1;
+          if (((c >> 1) & 7) >= 8 - kPolyPairsPvt) {
+            exp2_poly2(t0, t1, p0, p1);
+          } else {
+            p0 = ex2_approx(t0);
+            p1 = ex2_approx(t1);
+          }
           const int x = (c >> 1) & 3;
           add2(sa[x], sb[x], sa[x], sb[x], p0, p1);
           return pack_bf16x2(p0, p1);
@@ -1099,7 +1152,7 @@ __global__ void __launch_bounds__(384, 1)
         __nv_bfloat16* dst = a.part_o + static_cast<size_t>(prow) * D;
 #pragma unroll
         for (int c = 0; c < 16; ++c)
-          reinterpret_cast<uint4*>(dst)[c] = *reinterpret_cast<const uint4*>(sP + p_offset(q, c * 8));
+          st_part(reinterpret_cast<uint4*>(dst) + c, *reinterpret_cast<const uint4*>(sP + p_offset(q, c * 8)));
         a.part_lse[prow] = (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
       }
       // the P tile rows of this half are rewritten only by this warpgroup, after this point
@@ -1166,7 +1219,7 @@ cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream) {
   CUtensorMap mk, mv, mq;
   if (!make_kv_map(&mk, L.k, L.T, L.G, L.d) || !make_kv_map(&mv, L.v, L.T, L.G, L.d))
     return cudaErrorInvalidValue;
-  if (L.d == 64 && !make_q_rows_map(&mq, L.q, static_cast<long long>(L.T) * L.H, L.d))
+  if (!make_q_rows_map(&mq, L.q, static_cast<long long>(L.T) * L.H, L.d))
     return cudaErrorInvalidValue;
   AttnArgs a;
   a.q = static_cast<const __nv_bfloat16*>(L.q);
@@ -1209,7 +1262,7 @@ cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream) {
     const int smem = PvtCfg::SMEM_BYTES;
     cudaError_t e = cudaFuncSetAttribute(attn_kernel_pvt, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_kernel_pvt<<<grid, 384, smem, stream>>>(mk, mv, a);
+    attn_kernel_pvt<<<grid, 384, smem, stream>>>(mk, mv, mq, a);
   }
   return cudaGetLastError();
 }

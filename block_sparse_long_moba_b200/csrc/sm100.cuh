@@ -349,6 +349,13 @@ __device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, f
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
+__device__ __forceinline__ void sub2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n .reg .b64 a, b, d;\n mov.b64 a, {%2, %3};\n mov.b64 b, {%4, %5};\n"
+      " sub.rn.f32x2 d, a, b;\n mov.b64 {%0, %1}, d;\n}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // Orders later uses of a register after the preceding asm statement (e.g. tcgen05.wait::ld):
 // the empty asm redefines the value, so no use can be scheduled above it. Emits no instruction.
 __device__ __forceinline__ void reg_fence(uint32_t& x) { asm volatile("" : "+r"(x)); }
@@ -364,6 +371,29 @@ __device__ __forceinline__ float exp2_poly(float t) {
   const float f = __fadd_rn(t, -n);
   const float p = fmaf(fmaf(fmaf(0.05481659f, f, 0.24172845f), f, 0.6932464f), f, 0.9999938f);
   return __uint_as_float(__float_as_uint(p) + (__float_as_uint(r) << 23));
+}
+
+// exp2_poly for a pair of inputs with paired f32x2 instructions (same split and cubic): ten
+// instructions for two results, all on the FMA pipe except the two exponent insertions.
+__device__ __forceinline__ void exp2_poly2(float t0, float t1, float& p0, float& p1) {
+  t0 = fmaxf(t0, -120.f);
+  t1 = fmaxf(t1, -120.f);
+  float r0, r1, n0, n1, f0, f1, q0, q1;
+  add2(r0, r1, t0, t1, 12582912.f, 12582912.f);
+  sub2(n0, n1, r0, r1, 12582912.f, 12582912.f);
+  sub2(f0, f1, t0, t1, n0, n1);
+  fma2(q0, q1, 0.05481659f, 0.05481659f, f0, f1, 0.24172845f, 0.24172845f);
+  fma2(q0, q1, q0, q1, f0, f1, 0.6932464f, 0.6932464f);
+  fma2(q0, q1, q0, q1, f0, f1, 0.9999938f, 0.9999938f);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(r0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(r1) << 23));
+}
+
+// max of three fp32 values in one instruction (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
