@@ -1141,20 +1141,31 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int x = 0; x < 32; ++x) reg_fence(orr[x]);
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const int qq = half * kTile + c0 + x;
-          const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(orr[x]) * s_invl[qq]);
-          *reinterpret_cast<__nv_bfloat16*>(sP + p_offset(qq, row)) = b;
+        for (int x4 = 0; x4 < 32; x4 += 4) {
+          const int qq = half * kTile + c0 + x4;
+          const float4 il = *reinterpret_cast<const float4*>(s_invl + qq);
+          const float ilv[4] = {il.x, il.y, il.z, il.w};
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+            *reinterpret_cast<__nv_bfloat16*>(sP + p_offset(qq + x, row)) =
+                __float2bfloat16_rn(__uint_as_float(orr[x4 + x]) * ilv[x]);
         }
       }
       named_bar_sync(bar_id, 128);
-      if (valid) {
-        __nv_bfloat16* dst = a.part_o + static_cast<size_t>(prow) * D;
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          st_part(reinterpret_cast<uint4*>(dst) + c, *reinterpret_cast<const uint4*>(sP + p_offset(q, c * 8)));
-        a.part_lse[prow] = (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
+      // each warp writes its own 32 rows, two whole 256-byte rows per instruction (16 lanes each)
+      {
+        const int wrow0 = half * kTile + (warp & 3) * 32;
+        const int my_prow = valid ? prow : -1;
+        const int c = lane & 15;
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int rr = 2 * i + (lane >> 4);
+          const int pr = __shfl_sync(0xffffffffu, my_prow, rr);
+          const uint4 v = *reinterpret_cast<const uint4*>(sP + p_offset(wrow0 + rr, c * 8));
+          if (pr >= 0) st_part(reinterpret_cast<uint4*>(a.part_o + static_cast<size_t>(pr) * D) + c, v);
+        }
       }
+      if (valid) a.part_lse[prow] = (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
       // the P tile rows of this half are rewritten only by this warpgroup, after this point
       tc_fence_before();
     }
