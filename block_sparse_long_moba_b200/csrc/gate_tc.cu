@@ -265,17 +265,33 @@ __global__ void __launch_bounds__(256, 1)
         const int c0 = ch * C::CAP;
         const int n = min(C::CAP, i_max - c0);
         if (nchunks > 1 || p == 0) {
-          // split the fp32 centroids of blocks [c0, c0 + n) into hi / lo bf16 tiles
+          // split the fp32 centroids of blocks [c0, c0 + n) into hi / lo bf16 tiles; each thread
+          // issues the loads of four 8-column groups before converting any (latency-bound else)
           ok = __syncthreads_and(ok);
           const int nrows = (n + 15) & ~15;
-          for (int e = tid; ok && e < nrows * (D / 8); e += blockDim.x) {
-            const int rr = e / (D / 8), c8 = (e % (D / 8)) * 8;
-            uint4 hi = make_uint4(0, 0, 0, 0), lo = make_uint4(0, 0, 0, 0);
-            if (rr < n) {
-              const float4* src = reinterpret_cast<const float4*>(
-                  cents + (static_cast<size_t>(base + c0 + rr) * G + g) * D + c8);
-              const float4 a0 = __ldg(src), a1 = __ldg(src + 1);
-              const float x[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+          const int ngroups = nrows * (D / 8);
+          for (int e0 = tid; ok && e0 < ngroups; e0 += 4 * static_cast<int>(blockDim.x)) {
+            float4 va[4], vb[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int e = e0 + u * static_cast<int>(blockDim.x);
+              const int rr = e / (D / 8), c8 = (e % (D / 8)) * 8;
+              va[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+              vb[u] = va[u];
+              if (e < ngroups && rr < n) {
+                const float4* src = reinterpret_cast<const float4*>(
+                    cents + (static_cast<size_t>(base + c0 + rr) * G + g) * D + c8);
+                va[u] = __ldg(src);
+                vb[u] = __ldg(src + 1);
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int e = e0 + u * static_cast<int>(blockDim.x);
+              if (e >= ngroups) break;
+              const int rr = e / (D / 8), c8 = (e % (D / 8)) * 8;
+              const float x[8] = {va[u].x, va[u].y, va[u].z, va[u].w,
+                                  vb[u].x, vb[u].y, vb[u].z, vb[u].w};
               uint32_t hw[4], lw[4];
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
@@ -288,11 +304,11 @@ __global__ void __launch_bounds__(256, 1)
                 lw[k] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
                         (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
               }
-              hi = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-              lo = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+              *reinterpret_cast<uint4*>(smem + C::OFF_B + c_offset<D>(0, rr, c8)) =
+                  make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              *reinterpret_cast<uint4*>(smem + C::OFF_B + c_offset<D>(1, rr, c8)) =
+                  make_uint4(lw[0], lw[1], lw[2], lw[3]);
             }
-            *reinterpret_cast<uint4*>(smem + C::OFF_B + c_offset<D>(0, rr, c8)) = hi;
-            *reinterpret_cast<uint4*>(smem + C::OFF_B + c_offset<D>(1, rr, c8)) = lo;
           }
           fence_proxy_async_smem();
           __syncthreads();
