@@ -68,7 +68,7 @@ def gate_flops(w: wl.Workload) -> float:
 
 
 def kernel_bytes(w: wl.Workload) -> dict:
-    """Algorithmic HBM bytes per launch of the HBM-bound kernels (one chunk)."""
+    """Algorithmic HBM bytes of the HBM-bound kernels over one whole step (all query chunks)."""
     T, H, G, d, k = w.total_tokens, w.hq, w.hkv, w.d, w.topk
     NB = w.num_blocks
     routed = 0
@@ -385,7 +385,9 @@ def run_ours(args):
                 continue
             ent = {"ms_per_launch": kms / kn, "launches": kn, "share": kms / max(ms_local, 1e-9)}
             if name in kb:
-                gbs = kb[name] / (kms / kn / 1e3) / 1e9 / (1 if name != "merge" else 1)
+                # kb holds the bytes of one whole step; a chunked problem launches a kernel
+                # several times per step, so divide by the kernel's time per step
+                gbs = kb[name] / (kms / args.steps / 1e3) / 1e9
                 ent["gbs"] = gbs
                 ent["hbm_frac"] = gbs / peaks["hbm_gbs"]
             kern[name] = ent
