@@ -177,11 +177,15 @@ Layout layout_of(const Plan& P, int nseq, int Hq, int Hkv, int d, int topk) {
 template <class T>
 T* at(void* base, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(base) + off); }
 
-// The tensor-core gate keeps at most 32 past blocks per row in registers, so it serves topk <= 33;
-// larger topk uses the CUDA-core gate.
-cudaError_t run_gate(const void* q, const float* cents, const int32_t* cu_dev, int nseq, int max_nb,
-                     int T, int H, int G, int d, int B, int topk, int32_t* idx, int* status,
-                     int sms, cudaStream_t s) {
+// The tensor-core gates keep at most 32 past blocks per row in registers, so they serve
+// topk <= 33; larger topk uses the CUDA-core gate. Sequences of at most 257 blocks take the
+// streaming gate (all past centroids resident, query tiles streamed by a producer warp).
+cudaError_t run_gate(const void* q, const float* cents, const int32_t* cu_dev,
+                     const int32_t* cu_host, int nseq, int max_nb, int T, int H, int G, int d,
+                     int B, int topk, int32_t* idx, int* status, int sms, cudaStream_t s) {
+  if (gate_stream_supported(max_nb, topk))
+    return launch_gate_stream(q, cents, cu_dev, cu_host, nseq, max_nb, T, H, G, d, B, topk, idx,
+                              status, sms, s);
   if (topk <= 33)
     return launch_gate_tc(q, cents, cu_dev, nseq, max_nb, T, H, G, d, B, topk, idx, status, sms, s);
   return launch_gate(q, cents, cu_dev, nseq, max_nb, T, H, G, d, B, topk, idx, s);
@@ -258,8 +262,8 @@ int moba_gate_topk(const void* q, const float* centroids, const int32_t* cu_dev,
   if ((st = device_check(&sms)) != MOBA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   MOBA_LAUNCH(kGate, s,
-              run_gate(q, centroids, cu_dev, nseq, P.max_nb, P.T, Hq, Hkv, d, block_size, topk,
-                       block_idx, nullptr, sms, s));
+              run_gate(q, centroids, cu_dev, cu_host, nseq, P.max_nb, P.T, Hq, Hkv, d,
+                       block_size, topk, block_idx, nullptr, sms, s));
   return MOBA_OK;
 }
 
@@ -317,8 +321,8 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu
     MOBA_LAUNCH(kCentroid, s,
                 launch_centroids(k, cu_dev, nseq, P.max_nb, Hkv, d, block_size, P.NB, sms, cents, s));
     MOBA_LAUNCH(kGate, s,
-                run_gate(q, cents, cu_dev, nseq, P.max_nb, P.T, Hq, Hkv, d, block_size, topk, idx_w,
-                         status, sms, s));
+                run_gate(q, cents, cu_dev, cu_host, nseq, P.max_nb, P.T, Hq, Hkv, d, block_size,
+                         topk, idx_w, status, sms, s));
     idx = idx_w;
   } else if (block_idx_out && block_idx_out != block_idx_in) {
     if (cudaMemcpyAsync(block_idx_out, block_idx_in, static_cast<size_t>(Hq) * P.T * topk * 4,

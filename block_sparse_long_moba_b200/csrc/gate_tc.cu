@@ -1,25 +1,32 @@
-// K2 on the tensor cores — parameter-less causal top-k gate [MoBA paper summary (atlas.scime.ai),
-// "Approach"; MoBA README, "Parameter-less Gating Mechanism"].
+// K2 on the tensor cores, long-sequence form — parameter-less causal top-k gate [MoBA paper
+// summary (atlas.scime.ai), "Approach"; MoBA README, "Parameter-less Gating Mechanism"] for
+// sequences of more than 257 blocks (the small-block shapes: 512 to 1792 blocks of 128 keys).
 //
 // Scores of one tile of 128 query rows (128 consecutive tokens of one query head) against the past
 // blocks of their sequence are one matrix product on tcgen05:
 //   S[128, n] = Q[128, d] . C[n, d]^T,  C = c_hi + c_lo  (two bf16 terms of the fp32 centroids)
 // so each fp32 centroid enters with ~2^-17 relative error and every product q * c_part is exact
 // in the fp32 accumulator. The T x NB score matrix never exists in memory [FlashMoBA story,
-// FlashTopK]: up to 256 scores per row at a time live in tensor memory.
+// FlashTopK]: at most 256 scores per row at a time live in tensor memory, and the products are
+// recomputed for each pass below (the tensor pipe is otherwise idle here).
 //
-// Selection: one thread per row (= TMEM lane) keeps its running top list in registers, sorted
-// best first (strict comparison, so equal scores keep the lower block). Scores are read 32 at a
-// time; only when some row of the warp has a column that beats its current threshold are they
-// staged in shared memory, and each row then visits only those columns, so a warp pays for the
-// largest per-row candidate count of a chunk rather than for every column. An insertion computes
-// every position of the list independently (no compare-and-swap chain), so its cost is issue
-// slots rather than latency. Scores live in two 128-column TMEM buffers per warpgroup: the
-// products of the next 128 past blocks run on the tensor core while this piece is selected.
+// Selection, one thread per row (= TMEM lane), in three passes over the row's n scores:
+//   1. group maxima over M strided groups (column j in group j mod M, M = 32 or 64); the ksel-th
+//      largest group maximum tau is a lower bound of the ksel-th best score, since ksel distinct
+//      groups each hold a score >= tau;
+//   2. every score >= tau is a candidate (typically ksel + a few) and is appended to the row's
+//      candidate buffer in shared memory; a bitonic sort of the buffer gives the exact ksel-th
+//      best score tau* and how many of the selected scores tie with it;
+//   3. the columns with score > tau*, and the lowest-numbered ones equal to tau* (ties go to the
+//      lower block), are written out in ascending order.
+// Each pass costs a compare per score and no per-score list insertion; a single pass that keeps a
+// running top list pays an insertion for every score that beats the list's current threshold,
+// which is most of the early columns. A row whose candidates overflow the buffer (many exactly
+// equal scores) runs that single-pass selection in pass 3 instead.
 //
-// A CTA holds two warpgroups (one query tile each) and works on one (query block, kv head) unit at a
-// time: the split centroids of the unit's past blocks are converted into shared memory once and
-// reused by all r * B / 128 tiles of the unit when they fit, and streamed in chunks otherwise.
+// A CTA holds two warpgroups (one query tile each) and works on one (query blocks, kv head) unit
+// at a time: the split centroids of the unit's past blocks are converted into shared memory once
+// and reused by all tiles of the unit when they fit, and streamed in chunks otherwise.
 #include "common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
@@ -30,19 +37,24 @@ namespace {
 
 constexpr int kTilesPerUnit = 16;  // query tiles that share one conversion of the centroids
 
-template <int D>
+template <int D, int KCAP>
 struct GateCfg {
   static constexpr int NCB = D / 64;
+  static constexpr int M = (KCAP <= 16) ? 32 : 64;           // groups of pass 1
+  static constexpr int CB = (KCAP <= 16) ? 32 : 64;          // candidate slots per row
   static constexpr int Q_BYTES = kTile * D * 2;             // one 128-row query tile
-  static constexpr int CAP = (D == 128) ? 256 : 640;         // centroid rows resident at once
+  static constexpr int CAND_BYTES = 2 * CB * 128 * 4;        // [2][CB][128] fp32
+  // centroid rows resident at once: what is left of the CTA's shared memory
+  static constexpr int CAP = (D == 128) ? (KCAP <= 16 ? 256 : 192) : (KCAP <= 16 ? 640 : 512);
   static constexpr int B_BYTES = 2 * NCB * CAP * 128;        // hi + lo, 128 B per row per block
   static constexpr int OFF_B = 2 * Q_BYTES;                  // one Q buffer per warpgroup
-  static constexpr int OFF_STAGE = OFF_B + B_BYTES;          // [2][32][128] staged scores
-  static constexpr int OFF_BARS = OFF_STAGE + 2 * 32 * 128 * 4;
+  static constexpr int OFF_STAGE = OFF_B + B_BYTES;          // candidate buffer / staging
+  static constexpr int OFF_BARS = OFF_STAGE + CAND_BYTES;
   static constexpr int SMEM_BYTES = OFF_BARS + 256;
   static constexpr int PIECE = 128;                          // MMA N (scores per TMEM buffer)
 };
-static_assert(GateCfg<128>::SMEM_BYTES <= 232448 && GateCfg<64>::SMEM_BYTES <= 232448,
+static_assert(GateCfg<128, 16>::SMEM_BYTES <= 232448 && GateCfg<64, 16>::SMEM_BYTES <= 232448 &&
+                  GateCfg<128, 32>::SMEM_BYTES <= 232448 && GateCfg<64, 32>::SMEM_BYTES <= 232448,
               "shared memory budget of one CTA");
 
 struct GateBars {
@@ -52,30 +64,19 @@ struct GateBars {
   int red[32];
 };
 
-template <int D>
+template <int D, int KCAP>
 __device__ __forceinline__ uint32_t c_offset(int s, int row, int col) {
-  using C = GateCfg<D>;
+  using C = GateCfg<D, KCAP>;
   return static_cast<uint32_t>(s * C::NCB * C::CAP * 128 + (col >> 6) * C::CAP * 128) +
          sw128_offset(row, col & 63);
 }
 
-// Order-preserving map of fp32 to uint32 (a larger float gives a larger unsigned) and back.
-__device__ __forceinline__ uint32_t f2ord(float f) {
-  const uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float ord2f(uint32_t o) {
-  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
-}
-
-// Running top list of one row, best first. The first KCAP - ksel places hold sentinels that no
-// score displaces, so the last place is always the ksel-th best so far: the exact threshold.
-template <int KCAP, bool PACK>
-struct TopList;
-
-// Scores and block ids kept apart; equal scores keep the earlier (lower) block.
+// Running top list of one row (the single-pass selection that rows with overflowing candidate
+// buffers fall back to), best first. The first KCAP - ksel places hold sentinels that no score
+// displaces, so the last place is always the ksel-th best so far. Equal scores keep the earlier
+// (lower) block.
 template <int KCAP>
-struct TopList<KCAP, false> {
+struct TopList {
   float v[KCAP];
   int id[KCAP];
   __device__ __forceinline__ void init(int ksel) {
@@ -85,9 +86,7 @@ struct TopList<KCAP, false> {
       id[x] = 0x7fffffff;
     }
   }
-  // columns worth a closer look: s > thr with thr read once per 32 columns
   __device__ __forceinline__ float thr() const { return v[KCAP - 1]; }
-  __device__ __forceinline__ static bool cand(float s, float t) { return s > t; }
   // Inserts (s, j) if it beats the last place. gt[] is monotone (the list is sorted), so position
   // x takes the entry above it when s beats that one, s when s beats only the entry at x, and
   // keeps its entry otherwise: every position is computed independently.
@@ -104,46 +103,52 @@ struct TopList<KCAP, false> {
     v[0] = gt[0] ? s : v[0];
     id[0] = gt[0] ? j : id[0];
   }
-  __device__ __forceinline__ int block(int x) const { return id[x]; }
 };
 
-// One 32-bit key per entry, for sequences of at most 256 blocks: the order-preserving image of
-// the score with its low 8 bits replaced by 255 - block, so keys are distinct, a larger key is a
-// better score, and equal truncated scores rank the lower block first. The truncation changes an
-// order only between scores within 2^-15 of each other (relative), inside the near-tie band of the
-// routing rule. An insertion is then KCAP integer max and KCAP - 1 min operations.
-template <int KCAP>
-struct TopList<KCAP, true> {
-  uint32_t k[KCAP];
-  __device__ __forceinline__ void init(int ksel) {
+// Bitonic sorting network over N (a power of two) fp32 registers, descending.
+template <int N>
+__device__ __forceinline__ void bitonic_desc_f(float (&k)[N]) {
 #pragma unroll
-    for (int x = 0; x < KCAP; ++x) k[x] = (x < KCAP - ksel) ? 0xffffffffu : 0u;
-  }
-  // a key can only beat the last place if its score is at least this
-  __device__ __forceinline__ float thr() const {
-    return k[KCAP - 1] == 0u ? -INFINITY : ord2f(k[KCAP - 1] & ~0xffu);
-  }
-  __device__ __forceinline__ static bool cand(float s, float t) { return s >= t; }
-  __device__ __forceinline__ void offer(float s, int j) {
-    const uint32_t key = (f2ord(s) & ~0xffu) | static_cast<uint32_t>(255 - j);
-    if (key <= k[KCAP - 1]) return;
+  for (int size = 2; size <= N; size <<= 1) {
 #pragma unroll
-    for (int x = KCAP - 1; x > 0; --x) k[x] = max(k[x], min(k[x - 1], key));
-    k[0] = max(k[0], key);
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int a = 0; a < N; ++a) {
+        const int b = a ^ stride;
+        if (b > a) {
+          const float hi = fmaxf(k[a], k[b]), lo = fminf(k[a], k[b]);
+          if ((a & size) == 0) {
+            k[a] = hi;
+            k[b] = lo;
+          } else {
+            k[a] = lo;
+            k[b] = hi;
+          }
+        }
+      }
+    }
   }
-  __device__ __forceinline__ int block(int x) const {
-    return k[x] == 0xffffffffu ? 0x7fffffff : 255 - static_cast<int>(k[x] & 0xffu);
-  }
-};
+}
+
+// The smallest of the first ksel entries of a descending list: its ksel-th largest value.
+template <int N>
+__device__ __forceinline__ float kth_of_sorted(const float (&k)[N], int ksel) {
+  float t = INFINITY;
+#pragma unroll
+  for (int x = 0; x < N; ++x)
+    if (x < ksel) t = fminf(t, k[x]);
+  return t;
+}
 
 }  // namespace
 
-template <int D, int KCAP, bool PACK>
+template <int D, int KCAP>
 __global__ void __launch_bounds__(256, 1)
     gate_tc_kernel(const __grid_constant__ CUtensorMap map_q, const float* __restrict__ cents,
                    const int32_t* __restrict__ cu, int nseq, int max_nb, int T, int H, int G,
                    int B, int topk, int32_t* __restrict__ idx, int* __restrict__ status) {
-  using C = GateCfg<D>;
+  using C = GateCfg<D, KCAP>;
+  constexpr int M = C::M, CB = C::CB;
   extern __shared__ __align__(1024) uint8_t smem[];
   GateBars* bars = reinterpret_cast<GateBars*>(smem + C::OFF_BARS);
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -173,7 +178,8 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t tmem = bars->tmem_base;
   const uint32_t t_s = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + wg * 2 * C::PIECE;
   uint8_t* sQ = smem + wg * C::Q_BYTES;
-  float* stage = reinterpret_cast<float*>(smem + C::OFF_STAGE) + wg * 32 * 128;  // [x][row]
+  // this warpgroup's candidate buffer [CB][128] (pass 2), reused as staging [32][128] (pass 3)
+  float* cand = reinterpret_cast<float*>(smem + C::OFF_STAGE) + wg * CB * 128;
   const uint32_t sBa = smem_u32(smem + C::OFF_B);
   const int r = H / G;
   const int ksel = topk - 1;
@@ -192,12 +198,19 @@ __global__ void __launch_bounds__(256, 1)
   const int QG = max(1, kTilesPerUnit / tiles_per_block);      // query blocks per unit
   const int n_sub = (QG * tiles_per_block + kTilesPerUnit - 1) / kTilesPerUnit;
   const int n_groups = (max_nb + QG - 1) / QG;
-  const long long n_units = static_cast<long long>(nseq) * G * n_groups * n_sub;
-  for (long long u = blockIdx.x; u < n_units; u += gridDim.x) {
-    const int sub = static_cast<int>(u % n_sub);
-    long long rest = u / n_sub;
-    const int ig = static_cast<int>(rest % n_groups);
-    rest /= n_groups;
+  // Units are numbered heaviest first (query-block group ig descending: a later group scores
+  // more past blocks) and dealt to the CTAs in a snake order (0..grid-1, then grid-1..0, ...), so
+  // every CTA gets a similar mix of heavy and light units.
+  const long long per_ig = static_cast<long long>(nseq) * G * n_sub;
+  const long long n_units = per_ig * n_groups;
+  const long long grid = gridDim.x;
+  for (long long kr = 0;; ++kr) {
+    const long long u = kr * grid + ((kr & 1) ? grid - 1 - blockIdx.x : blockIdx.x);
+    if (u >= n_units) break;
+    const int ig = n_groups - 1 - static_cast<int>(u / per_ig);
+    long long rest = u % per_ig;
+    const int sub = static_cast<int>(rest % n_sub);
+    rest /= n_sub;
     const int g = static_cast<int>(rest % G);
     const int s = static_cast<int>(rest / G);
     const int seq0 = cu[s], L = cu[s + 1] - seq0;
@@ -251,172 +264,251 @@ __global__ void __launch_bounds__(256, 1)
       int i_t = 0, h = 0, t0 = 0, rows = 0;
       if (tile < ntiles) tile_info(tile, i_t, h, t0, rows);
       const bool scored = tile < ntiles && rows > 0 && i_t > ksel && ksel > 0;
+      int32_t* out = idx + (static_cast<size_t>(h) * T + t0 + row) * topk;
       if (tile < ntiles && rows > 0 && !scored && row < rows) {
         // few causal blocks or topk == 1: the selection is fixed, no scores needed
-        int32_t* out = idx + (static_cast<size_t>(h) * T + t0 + row) * topk;
         if (ksel == 0) out[0] = i_t;
         else
           for (int x = 0; x < topk; ++x) out[x] = (x <= i_t) ? x : -1;
       }
-      TopList<KCAP, PACK> top;
+      // per-row selection state across the three passes
+      float gmax[M];
+#pragma unroll
+      for (int x = 0; x < M; ++x) gmax[x] = -INFINITY;
+      float tau = -INFINITY, tau_star = INFINITY;
+      int cnt = 0, tie_budget = 0, pos = 0;
+      bool overflow = false;
+      TopList<KCAP> top;
       top.init(ksel);
       bool q_ready = false;
-      for (int ch = 0; ch < nchunks; ++ch) {
-        const int c0 = ch * C::CAP;
-        const int n = min(C::CAP, i_max - c0);
-        if (nchunks > 1 || p == 0) {
-          // split the fp32 centroids of blocks [c0, c0 + n) into hi / lo bf16 tiles; each thread
-          // issues the loads of four 8-column groups before converting any (latency-bound else)
-          ok = __syncthreads_and(ok);
-          const int nrows = (n + 15) & ~15;
-          const int ngroups = nrows * (D / 8);
-          for (int e0 = tid; ok && e0 < ngroups; e0 += 4 * static_cast<int>(blockDim.x)) {
-            float4 va[4], vb[4];
+      for (int pass = 0; pass < 3; ++pass) {
+        for (int ch = 0; ch < nchunks; ++ch) {
+          const int c0 = ch * C::CAP;
+          const int n = min(C::CAP, i_max - c0);
+          if (nchunks > 1 || (p == 0 && pass == 0)) {
+            // split the fp32 centroids of blocks [c0, c0 + n) into hi / lo bf16 tiles; each thread
+            // issues the loads of eight 8-column groups before converting any
+            ok = __syncthreads_and(ok);
+            const int nrows = (n + 15) & ~15;
+            const int ngroups = nrows * (D / 8);
+            for (int e0 = tid; ok && e0 < ngroups; e0 += 8 * static_cast<int>(blockDim.x)) {
+              float4 va[8], vb[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int e = e0 + u * static_cast<int>(blockDim.x);
-              const int rr = e / (D / 8), c8 = (e % (D / 8)) * 8;
-              va[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-              vb[u] = va[u];
-              if (e < ngroups && rr < n) {
-                const float4* src = reinterpret_cast<const float4*>(
-                    cents + (static_cast<size_t>(base + c0 + rr) * G + g) * D + c8);
-                va[u] = __ldg(src);
-                vb[u] = __ldg(src + 1);
+              for (int uu = 0; uu < 8; ++uu) {
+                const int e = e0 + uu * static_cast<int>(blockDim.x);
+                const int rr = e / (D / 8), c8 = (e % (D / 8)) * 8;
+                va[uu] = make_float4(0.f, 0.f, 0.f, 0.f);
+                vb[uu] = va[uu];
+                if (e < ngroups && rr < n) {
+                  const float4* src = reinterpret_cast<const float4*>(
+                      cents + (static_cast<size_t>(base + c0 + rr) * G + g) * D + c8);
+                  va[uu] = __ldg(src);
+                  vb[uu] = __ldg(src + 1);
+                }
+              }
+#pragma unroll
+              for (int uu = 0; uu < 8; ++uu) {
+                const int e = e0 + uu * static_cast<int>(blockDim.x);
+                if (e >= ngroups) break;
+                const int rr = e / (D / 8), c8 = (e % (D / 8)) * 8;
+                const float x[8] = {va[uu].x, va[uu].y, va[uu].z, va[uu].w,
+                                    vb[uu].x, vb[uu].y, vb[uu].z, vb[uu].w};
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * k]);
+                  const __nv_bfloat16 h1 = __float2bfloat16_rn(x[2 * k + 1]);
+                  const __nv_bfloat16 l0 = __float2bfloat16_rn(x[2 * k] - __bfloat162float(h0));
+                  const __nv_bfloat16 l1 =
+                      __float2bfloat16_rn(x[2 * k + 1] - __bfloat162float(h1));
+                  hw[k] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                          (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+                  lw[k] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
+                          (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+                }
+                *reinterpret_cast<uint4*>(smem + C::OFF_B + c_offset<D, KCAP>(0, rr, c8)) =
+                    make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4*>(smem + C::OFF_B + c_offset<D, KCAP>(1, rr, c8)) =
+                    make_uint4(lw[0], lw[1], lw[2], lw[3]);
               }
             }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int e = e0 + u * static_cast<int>(blockDim.x);
-              if (e >= ngroups) break;
-              const int rr = e / (D / 8), c8 = (e % (D / 8)) * 8;
-              const float x[8] = {va[u].x, va[u].y, va[u].z, va[u].w,
-                                  vb[u].x, vb[u].y, vb[u].z, vb[u].w};
-              uint32_t hw[4], lw[4];
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * k]);
-                const __nv_bfloat16 h1 = __float2bfloat16_rn(x[2 * k + 1]);
-                const __nv_bfloat16 l0 = __float2bfloat16_rn(x[2 * k] - __bfloat162float(h0));
-                const __nv_bfloat16 l1 = __float2bfloat16_rn(x[2 * k + 1] - __bfloat162float(h1));
-                hw[k] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
-                        (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
-                lw[k] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
-                        (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
-              }
-              *reinterpret_cast<uint4*>(smem + C::OFF_B + c_offset<D>(0, rr, c8)) =
-                  make_uint4(hw[0], hw[1], hw[2], hw[3]);
-              *reinterpret_cast<uint4*>(smem + C::OFF_B + c_offset<D>(1, rr, c8)) =
-                  make_uint4(lw[0], lw[1], lw[2], lw[3]);
-            }
+            fence_proxy_async_smem();
+            __syncthreads();
           }
-          fence_proxy_async_smem();
-          __syncthreads();
-        }
-        if (!scored || c0 >= i_t) continue;  // warpgroup-uniform
-        const int n_t = min(n, i_t - c0);       // this tile's past blocks in the chunk
-        if (!q_ready) {
-          const bool w = ok && mbar_wait_bounded(&bars->q_full[wg], qphase, abort_flag, status,
-                                                 kDevTimeoutAttn, TO);
-          qphase ^= 1;
-          q_ready = true;
-          ok = named_bar_and(1 + wg, 128, w);
-        }
-        // scores of this chunk, 128 past blocks per TMEM buffer; the products of piece p + 1 are
-        // issued before piece p is selected (its buffer was freed by the barrier ending p - 1)
-        const uint32_t qa = smem_u32(sQ);
-        auto issue = [&](int p0) {  // one converged warp of the warpgroup issues
-          const int nmma = (min(C::PIECE, n_t - p0) + 15) & ~15;
-          const uint32_t idesc = idesc_bf16_f32(128, nmma, 0, 0);
-          const uint32_t buf = npiece & 1;
-          tc_fence_after();
-#pragma unroll
-          for (int sp = 0; sp < 2; ++sp) {
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-              const uint32_t aoff = (ks >> 2) * 16384 + (ks & 3) * 32;
-              const uint32_t boff = static_cast<uint32_t>(sp * C::NCB * C::CAP * 128 +
-                                                          (ks >> 2) * C::CAP * 128 + p0 * 128 +
-                                                          (ks & 3) * 32);
-              mma_ss_elect(tmem + wg * 2 * C::PIECE + buf * C::PIECE,
-                           smem_desc_sw128(qa + aoff, 16, 1024),
-                           smem_desc_sw128(sBa + boff, 16, 1024), idesc,
-                           (sp > 0 || ks > 0) ? 1u : 0u);
-            }
+          if (!scored || c0 >= i_t) continue;  // warpgroup-uniform
+          const int n_t = min(n, i_t - c0);       // this tile's past blocks in the chunk
+          if (!q_ready) {
+            const bool w = ok && mbar_wait_bounded(&bars->q_full[wg], qphase, abort_flag, status,
+                                                   kDevTimeoutAttn, TO);
+            qphase ^= 1;
+            q_ready = true;
+            ok = named_bar_and(1 + wg, 128, w);
           }
-          mma_commit_elect(&bars->mma_done[wg][buf]);
-        };
-        if (ok && warp == wg * 4) issue(0);
-        ++npiece;
-        for (int p0 = 0; p0 < n_t; p0 += C::PIECE) {
-          const int np = min(C::PIECE, n_t - p0);
-          const uint32_t pc = npiece - 1;  // this piece's number
-          if (p0 + C::PIECE < n_t) {
-            if (ok && warp == wg * 4) issue(p0 + C::PIECE);
-            ++npiece;
-          }
-          const bool w = ok && mbar_wait_bounded(&bars->mma_done[wg][pc & 1], (pc >> 1) & 1,
-                                                 abort_flag, status, kDevTimeoutAttn, TO);
-          // the Q buffer is free once the tile's last product is done: fetch the next one
-          const bool last_pass = (c0 + n >= i_t || ch == nchunks - 1) && p0 + C::PIECE >= n_t;
-          if (row == 0 && w && last_pass) {
-            const int t = next_scored(tile + 2);
-            if (t < ntiles) load_q(t);
-          }
-          if (__all_sync(0xffffffffu, w)) {
+          // scores of this chunk, 128 past blocks per TMEM buffer; the products of piece p + 1 are
+          // issued before piece p is selected (its buffer was freed by the barrier ending p - 1)
+          const uint32_t qa = smem_u32(sQ);
+          auto issue = [&](int p0) {  // one converged warp of the warpgroup issues
+            const int nmma = (min(C::PIECE, n_t - p0) + 15) & ~15;
+            const uint32_t idesc = idesc_bf16_f32(128, nmma, 0, 0);
+            const uint32_t buf = npiece & 1;
             tc_fence_after();
-            const uint32_t tb = t_s + (pc & 1) * C::PIECE;
-            for (int cc = 0; cc < np; cc += 32) {
-              uint32_t sr[32];
-              tmem_ld32(tb + cc, sr);
-              tmem_wait_ld();
 #pragma unroll
-              for (int x = 0; x < 32; ++x) reg_fence(sr[x]);
-              // candidates: columns that beat this row's current threshold
-              const float thr0 = top.thr();
-              uint32_t mask = 0;
+            for (int sp = 0; sp < 2; ++sp) {
 #pragma unroll
-              for (int x = 0; x < 32; ++x)
-                if (cc + x < np && top.cand(__uint_as_float(sr[x]), thr0)) mask |= 1u << x;
-              if (__any_sync(0xffffffffu, mask != 0)) {
-                // stage this thread's scores so that a candidate can be picked by its column
+              for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t aoff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                const uint32_t boff = static_cast<uint32_t>(sp * C::NCB * C::CAP * 128 +
+                                                            (ks >> 2) * C::CAP * 128 + p0 * 128 +
+                                                            (ks & 3) * 32);
+                mma_ss_elect(tmem + wg * 2 * C::PIECE + buf * C::PIECE,
+                             smem_desc_sw128(qa + aoff, 16, 1024),
+                             smem_desc_sw128(sBa + boff, 16, 1024), idesc,
+                             (sp > 0 || ks > 0) ? 1u : 0u);
+              }
+            }
+            mma_commit_elect(&bars->mma_done[wg][buf]);
+          };
+          if (ok && warp == wg * 4) issue(0);
+          ++npiece;
+          for (int p0 = 0; p0 < n_t; p0 += C::PIECE) {
+            const int np = min(C::PIECE, n_t - p0);
+            const uint32_t pc = npiece - 1;  // this piece's number
+            if (p0 + C::PIECE < n_t) {
+              if (ok && warp == wg * 4) issue(p0 + C::PIECE);
+              ++npiece;
+            }
+            const bool w = ok && mbar_wait_bounded(&bars->mma_done[wg][pc & 1], (pc >> 1) & 1,
+                                                   abort_flag, status, kDevTimeoutAttn, TO);
+            // the Q buffer is free once the tile's last product of the last pass is done
+            const bool last_pass = pass == 2 && (c0 + n >= i_t || ch == nchunks - 1) &&
+                                   p0 + C::PIECE >= n_t;
+            if (row == 0 && w && last_pass) {
+              const int t = next_scored(tile + 2);
+              if (t < ntiles) load_q(t);
+            }
+            if (__all_sync(0xffffffffu, w)) {
+              tc_fence_after();
+              const uint32_t tb = t_s + (pc & 1) * C::PIECE;
+              for (int cc = 0; cc < np; cc += 32) {
+                uint32_t sr[32];
+                tmem_ld32(tb + cc, sr);
+                tmem_wait_ld();
 #pragma unroll
-                for (int x = 0; x < 32; ++x) stage[x * 128 + row] = __uint_as_float(sr[x]);
-                const int jb = c0 + p0 + cc;
-                while (__any_sync(0xffffffffu, mask != 0)) {
-                  if (mask) {
-                    const int x = __ffs(mask) - 1;
-                    mask &= mask - 1;
-                    top.offer(stage[x * 128 + row], jb + x);
+                for (int x = 0; x < 32; ++x) reg_fence(sr[x]);
+                const int jb = c0 + p0 + cc;  // block of column x is jb + x (jb % 32 == 0)
+                if (pass == 0) {
+                  // group maxima, column j in group j mod M
+                  if (M == 32 || (jb & 32) == 0) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x)
+                      if (cc + x < np) gmax[x] = fmaxf(gmax[x], __uint_as_float(sr[x]));
+                  } else {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x)
+                      if (cc + x < np)
+                        gmax[(32 + x) % M] = fmaxf(gmax[(32 + x) % M], __uint_as_float(sr[x]));
+                  }
+                } else if (pass == 1) {
+                  // every score >= tau is a candidate
+#pragma unroll
+                  for (int x = 0; x < 32; ++x) {
+                    const float sv = __uint_as_float(sr[x]);
+                    if (cc + x < np && sv >= tau) {
+                      if (cnt < CB) cand[cnt * 128 + row] = sv;
+                      ++cnt;
+                    }
+                  }
+                } else {
+                  if (!overflow) {
+                    // columns above tau*, and the lowest-numbered ties while the budget lasts
+                    uint32_t gtm = 0, eqm = 0;
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) {
+                      const float sv = __uint_as_float(sr[x]);
+                      if (cc + x < np) {
+                        if (sv > tau_star) gtm |= 1u << x;
+                        else if (sv == tau_star) eqm |= 1u << x;
+                      }
+                    }
+                    while (__popc(eqm) > tie_budget) eqm &= ~(1u << (31 - __clz(eqm)));
+                    tie_budget -= __popc(eqm);
+                    uint32_t m = gtm | eqm;
+                    while (m) {
+                      const int x = __ffs(m) - 1;
+                      m &= m - 1;
+                      if (row < rows) out[pos] = jb + x;
+                      ++pos;
+                    }
+                  }
+                  // rows whose candidates overflowed keep a running top list instead
+                  const float thr0 = top.thr();
+                  uint32_t mask = 0;
+                  if (overflow) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x)
+                      if (cc + x < np && __uint_as_float(sr[x]) > thr0) mask |= 1u << x;
+                  }
+                  if (__any_sync(0xffffffffu, mask != 0)) {
+                    if (overflow) {
+#pragma unroll
+                      for (int x = 0; x < 32; ++x) cand[x * 128 + row] = __uint_as_float(sr[x]);
+                    }
+                    while (__any_sync(0xffffffffu, mask != 0)) {
+                      if (mask) {
+                        const int x = __ffs(mask) - 1;
+                        mask &= mask - 1;
+                        top.offer(cand[x * 128 + row], jb + x);
+                      }
+                    }
+                    __syncwarp();
                   }
                 }
-                __syncwarp();
               }
+              tc_fence_before();
             }
-            tc_fence_before();
+            // every thread of the warpgroup has read this buffer before piece p + 2 overwrites it
+            ok = named_bar_and(1 + wg, 128, w);
           }
-          // every thread of the warpgroup has read this buffer before piece p + 2 overwrites it
-          ok = named_bar_and(1 + wg, 128, w);
+        }
+        if (!scored) continue;
+        if (pass == 0) {
+          // tau: the ksel-th largest group maximum (ksel <= M groups hold a score >= tau)
+          bitonic_desc_f<M>(gmax);
+          tau = kth_of_sorted<M>(gmax, ksel);
+        } else if (pass == 1) {
+          overflow = cnt > CB;
+          if (!overflow) {
+            float cv[CB];
+#pragma unroll
+            for (int x = 0; x < CB; ++x) cv[x] = (x < cnt) ? cand[x * 128 + row] : -INFINITY;
+            bitonic_desc_f<CB>(cv);
+            tau_star = kth_of_sorted<CB>(cv, ksel);
+            int above = 0;
+#pragma unroll
+            for (int x = 0; x < CB; ++x) above += (cv[x] > tau_star) ? 1 : 0;
+            tie_budget = ksel - above;
+          }
         }
       }
       if (!scored || row >= rows || !ok) continue;
-      // the ksel real entries (sentinels map to INT_MAX), ascending
-      int sel[KCAP];
+      if (overflow) {
+        // the ksel real entries of the running list (sentinels map to INT_MAX), ascending
+        int sel[KCAP];
 #pragma unroll
-      for (int x = 0; x < KCAP; ++x) sel[x] = top.block(x);
+        for (int x = 0; x < KCAP; ++x) sel[x] = top.id[x];
 #pragma unroll
-      for (int a0 = 0; a0 < KCAP - 1; ++a0) {
+        for (int a0 = 0; a0 < KCAP - 1; ++a0) {
 #pragma unroll
-        for (int b0 = 0; b0 < KCAP - 1 - a0; ++b0) {
-          const int lo_ = min(sel[b0], sel[b0 + 1]), hi_ = max(sel[b0], sel[b0 + 1]);
-          sel[b0] = lo_;
-          sel[b0 + 1] = hi_;
+          for (int b0 = 0; b0 < KCAP - 1 - a0; ++b0) {
+            const int lo_ = min(sel[b0], sel[b0 + 1]), hi_ = max(sel[b0], sel[b0 + 1]);
+            sel[b0] = lo_;
+            sel[b0 + 1] = hi_;
+          }
         }
-      }
-      int32_t* out = idx + (static_cast<size_t>(h) * T + t0 + row) * topk;
 #pragma unroll
-      for (int x = 0; x < KCAP; ++x)
-        if (x < ksel) out[x] = sel[x];
+        for (int x = 0; x < KCAP; ++x)
+          if (x < ksel) out[x] = sel[x];
+      }
       out[ksel] = i_t;
     }
     ok = __syncthreads_and(ok);
@@ -458,29 +550,17 @@ bool make_q_map(CUtensorMap* map, const void* q, int T, int H, int D) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int KCAP, bool PACK>
-cudaError_t launch_tp(const CUtensorMap& mq, const float* cents, const int32_t* cu, int nseq,
-                      int max_nb, int T, int H, int G, int B, int topk, int32_t* idx, int* status,
-                      int grid, cudaStream_t stream) {
-  const int smem = GateCfg<D>::SMEM_BYTES;
-  cudaError_t e = cudaFuncSetAttribute(gate_tc_kernel<D, KCAP, PACK>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  gate_tc_kernel<D, KCAP, PACK><<<grid, 256, smem, stream>>>(mq, cents, cu, nseq, max_nb, T, H,
-                                                             G, B, topk, idx, status);
-  return cudaGetLastError();
-}
-
-// Packed keys need every block id of a sequence to fit in 8 bits.
 template <int D, int KCAP>
 cudaError_t launch_t(const CUtensorMap& mq, const float* cents, const int32_t* cu, int nseq,
                      int max_nb, int T, int H, int G, int B, int topk, int32_t* idx, int* status,
                      int grid, cudaStream_t stream) {
-  if (max_nb <= 256)
-    return launch_tp<D, KCAP, true>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status,
-                                    grid, stream);
-  return launch_tp<D, KCAP, false>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status,
-                                   grid, stream);
+  const int smem = GateCfg<D, KCAP>::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(gate_tc_kernel<D, KCAP>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  gate_tc_kernel<D, KCAP><<<grid, 256, smem, stream>>>(mq, cents, cu, nseq, max_nb, T, H, G, B,
+                                                       topk, idx, status);
+  return cudaGetLastError();
 }
 
 template <int D>

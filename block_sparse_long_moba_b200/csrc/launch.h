@@ -18,6 +18,26 @@ cudaError_t launch_gate(const void* q, const float* cents, const int32_t* cu_dev
                         int max_nb, int T, int H, int G, int d, int B, int topk, int32_t* idx,
                         cudaStream_t stream);
 
+// Per-CTA starts of the streaming gate's tile ranges (host-computed, passed by value).
+constexpr int kGateMaxCtas = 160;
+struct GateSched {
+  int n_cta;
+  int seg[kGateMaxCtas];    // s * Hkv + g of the first tile
+  int blk[kGateMaxCtas];    // its local block i
+  int pos[kGateMaxCtas];    // its index inside the block: head-in-group * tiles(i) + piece
+  int base[kGateMaxCtas];   // first global block of its sequence
+  int count[kGateMaxCtas];  // tiles of the range
+};
+
+// Streaming tensor-core gate for sequences of at most 257 blocks and topk <= 33.
+bool gate_stream_supported(int max_nb, int topk);
+int gate_stream_schedule(const int32_t* cu_host, int nseq, int H, int G, int d, int B, int topk,
+                         int num_ctas, GateSched* S);
+cudaError_t launch_gate_stream(const void* q, const float* cents, const int32_t* cu_dev,
+                               const int32_t* cu_host, int nseq, int max_nb, int T, int H, int G,
+                               int d, int B, int topk, int32_t* idx, int* status, int num_sms,
+                               cudaStream_t stream);
+
 // Tensor-core gate (scores on tcgen05, top-k in registers). `status` may be null.
 cudaError_t launch_gate_tc(const void* q, const float* cents, const int32_t* cu_dev, int nseq,
                            int max_nb, int T, int H, int G, int d, int B, int topk, int32_t* idx,

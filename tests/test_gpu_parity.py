@@ -55,6 +55,9 @@ def test_centroids_match_oracle(moba, cu, hkv, d, B):
     ([0, 2048], 2, 1, 128, 128, 1, "offset"),
     ([0, 6144], 2, 2, 64, 64, 40, "clusters"),          # topk above the buffered-selection limit
     ([0, 20000, 20000, 40000], 2, 1, 128, 64, 33, "clusters"),  # > 256 past blocks: chunked
+    ([0, 40000], 2, 2, 64, 128, 16, "clusters"),        # 313 blocks: three-pass selection
+    ([0, 33000, 33000, 70000], 2, 2, 64, 128, 32, "clusters"),  # 258 and 290 blocks, k - 1 = 31
+    ([0, 90000], 2, 1, 64, 128, 8, "offset"),           # 704 blocks: centroids in two chunks
 ])
 def test_gate_matches_oracle(moba, cu, hq, hkv, d, B, topk, keys):
     w, q, k, v, cu_t = _inputs(cu, hq, hkv, d, B, topk, keys)
@@ -64,6 +67,28 @@ def test_gate_matches_oracle(moba, cu, hq, hkv, d, B, topk, keys):
     cents = ref.centroids(k.cpu(), cu, B)
     tokens = np.arange(cu[-1])
     pu.check_routing(q.cpu(), cents, cu, B, topk, tokens, idx.cpu().numpy())
+
+
+@pytest.mark.parametrize("nblocks,topk", [(100, 12), (300, 16), (300, 32)])
+def test_gate_equal_scores_take_lowest_blocks(moba, nblocks, topk):
+    """All keys equal, so every past block scores the same: ties go to the lower block, so each
+    row routes to blocks 0 .. topk - 2 and its own (the single-pass and three-pass selections,
+    including the candidate-overflow fallback, all keep that order)."""
+    B = 128
+    T = nblocks * B
+    cu = [0, T]
+    q = torch.randn(T, 2, 64, device="cuda").to(torch.bfloat16)
+    k = torch.full((T, 2, 64), 0.5, device="cuda", dtype=torch.bfloat16)
+    cu_t = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    c = moba.moba_centroids(k, cu_t, cu, B)
+    idx = moba.moba_gate_topk(q, c, cu_t, cu, B, topk).cpu()
+    i = torch.arange(T) // B
+    expect = torch.full((T, topk), -1, dtype=torch.int32)
+    for x in range(topk):
+        expect[:, x] = torch.where(x < torch.clamp(i, max=topk - 1), x, -1)
+    n_sel = torch.clamp(i + 1, max=topk)
+    expect[torch.arange(T), n_sel - 1] = i.to(torch.int32)
+    assert torch.equal(idx[0], expect) and torch.equal(idx[1], expect)
 
 
 # ----------------------------------------------------------------------- whole forward, small
