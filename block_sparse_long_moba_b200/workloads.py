@@ -69,6 +69,8 @@ WORKLOADS = {
     # small cases of the same kernels for profiler captures (a few GB on the device)
     "profile_32k_b4096": Workload("profile_32k_b4096", [0, 32768], 32, 8, 128, 4096, 4, "offset"),
     "profile_32k_b128": Workload("profile_32k_b128", [0, 32768], 16, 16, 64, 128, 16, "clusters"),
+    # the gate's 256-block regime of the 1M shape (n up to 255 past blocks, k - 1 = 11) at 1 GB of Q
+    "profile_128k_b512": Workload("profile_128k_b512", [0, 131072], 32, 8, 128, 512, 12, "offset"),
 }
 WORKLOAD_ORDER = ["tiny_1k", "llama8b_128k", "llama8b_1m", "routing_64k_b128", "varlen_512k_b128"]
 

@@ -38,6 +38,12 @@ def _inputs(cu, hq, hkv, d, B, topk, keys="offset", seed=0):
     ([0, 1024], 1, 64, 128),
     ([0, 300, 300, 1000, 1100], 4, 128, 64),   # ragged tails, empty sequence, short sequence
     ([0, 8192], 8, 128, 4096),
+    # at least 74 blocks: whole-row form
+    ([0, 5000, 5000, 12000], 3, 64, 64),          # rows of 24 pieces: 10 rows per pass
+    ([0, 10000], 32, 128, 128),                    # rows of 512 pieces: two per thread
+    ([0, 9600], 64, 128, 128),                     # rows of 1024 pieces: four per thread
+    ([0, 4800], 72, 128, 64),                      # wider rows: one kv head per cluster
+    ([0, 65536], 16, 64, 128),                     # the 128-key-block shape
 ])
 def test_centroids_match_oracle(moba, cu, hkv, d, B):
     w, q, k, v, cu_t = _inputs(cu, hkv, hkv, d, B, 2)
