@@ -91,6 +91,8 @@ def kernel_bytes(w: wl.Workload) -> dict:
         "route_count": T * H * k * 4,
         "route_scatter": T * H * k * 4 + routed * 4,
         "merge": slots * (2 * d + 4) + T * H * (2 * d + 4),
+        # d = 64: each routed entry is read (4 B), its query row read and written (2 d B each)
+        **({"densify": routed * (4 + 4 * d)} if d == 64 else {}),
     }
 
 

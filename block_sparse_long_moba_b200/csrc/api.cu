@@ -17,8 +17,10 @@ using namespace moba;
 namespace {
 
 constexpr size_t kPartialBudgetBytes = 16ull << 30;  // per-chunk partial outputs + routing lists
-constexpr int kNumClasses = 8;
-enum KernelClass { kCentroid = 0, kGate, kRouteCount, kRouteScan, kRouteScatter, kAttn, kMerge, kPlan };
+constexpr int kNumClasses = 9;
+enum KernelClass {
+  kCentroid = 0, kGate, kRouteCount, kRouteScan, kRouteScatter, kAttn, kMerge, kPlan, kDensify
+};
 
 std::atomic<long long> g_launches{0};
 
@@ -118,7 +120,10 @@ int make_plan(int nseq, const int32_t* cu, int Hq, int Hkv, int d, int B, int to
   if (static_cast<long long>(P->T) * Hq >= (1LL << 31) / 2) return MOBA_ERR_UNSUPPORTED;
   if (P->max_nb > 65535) return MOBA_ERR_UNSUPPORTED;
   // query chunks of whole blocks, so that partial rows (t, h, slot) fit the budget
-  const size_t row_bytes = static_cast<size_t>(d) * 2 + 4 + 4;
+  // per partial row: its bf16 output, log-sum-exp and routing entry; at d = 64 also the copy of
+  // the routed query row that the attention kernel reads as a dense tile
+  const size_t row_bytes =
+      static_cast<size_t>(d) * 2 + 4 + 4 + (d == 64 ? static_cast<size_t>(d) * 2 : 0);
   size_t max_rows = std::max<size_t>(partial_budget / row_bytes, 1);
   const size_t per_tok = static_cast<size_t>(Hq) * topk;
   max_rows = std::min<size_t>(max_rows, (1ull << 31) - 1);
@@ -148,7 +153,7 @@ int make_plan(int nseq, const int32_t* cu, int Hq, int Hkv, int d, int B, int to
 // --------------------------------------------------------------------------- workspace carve
 struct Layout {
   size_t status, blk_off, blk_seq, blk_start, blk_len, cents, idx, counts, cursor, tiles,
-      entries, part_o, part_lse, total;
+      entries, qdense, part_o, part_lse, total;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -168,6 +173,7 @@ Layout layout_of(const Plan& P, int nseq, int Hq, int Hkv, int d, int topk) {
   L.cursor = take(static_cast<size_t>(Hkv) * P.NB * 4);
   L.tiles = take(P.max_tiles * 16);
   L.entries = take(std::max<size_t>(P.max_entries, 1) * 4);
+  L.qdense = take(d == 64 ? std::max<size_t>(P.max_entries, 1) * d * 2 : 0);
   L.part_o = take(P.max_rows * d * 2);
   L.part_lse = take(P.max_rows * 4);
   L.total = o;
@@ -311,6 +317,7 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu
   void* part_o = at<void>(workspace, L.part_o);
   float* part_lse = at<float>(workspace, L.part_lse);
   float* cents = at<float>(workspace, L.cents);
+  void* qdense = (d == 64) ? at<void>(workspace, L.qdense) : nullptr;
   const int NBK = Hkv * P.NB;
 
   MOBA_LAUNCH(kPlan, s, launch_plan(cu_dev, nseq, block_size, P.NB, tb, counts, NBK, status, s));
@@ -338,9 +345,15 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu
     MOBA_LAUNCH(kRouteScatter, s,
                 launch_route_scatter(idx, tb, P.T, Hq, Hkv, topk, P.NB, c.b0, c.nblk, c.T0,
                                      P.max_nb, cursor, entries, s));
+    if (qdense)
+      MOBA_LAUNCH(kDensify, s,
+                  launch_densify(entries, n_tiles + 1, q, Hq, topk, c.T0,
+                                 static_cast<long long>(P.max_entries), qdense, sms, s));
     AttnLaunch A;
     A.q = q; A.k = k; A.v = v;
     A.tiles = tiles; A.n_routed = n_tiles; A.entries = entries; A.tb = tb;
+    A.qdense = qdense;
+    A.qdense_rows = static_cast<long long>(std::max<size_t>(P.max_entries, 1));
     A.part_o = part_o; A.part_lse = part_lse; A.status = status;
     A.T = P.T; A.H = Hq; A.G = Hkv; A.d = d; A.B = block_size; A.topk = topk; A.NB = P.NB;
     A.b0 = c.b0; A.nblk = c.nblk; A.T0 = c.T0; A.scale = scale;

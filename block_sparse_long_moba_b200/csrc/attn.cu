@@ -210,11 +210,12 @@ struct D64Cfg {
   static constexpr int D = 64;
   static constexpr int HALF_BYTES = kTile * D * 2;  // 16 KB: one 128 x 64 bf16 tile
   static constexpr int Q_BYTES = 2 * HALF_BYTES;    // one 256-row item
-  static constexpr int QB = 4;                      // Q buffers (items gathered ahead)
+  static constexpr int QB = 3;                      // Q buffers (items loaded ahead)
   static constexpr int NK = 2, NV = 3;              // K and V ring depths (V is freed later)
   static constexpr int OFF_K = QB * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NK * HALF_BYTES;
-  static constexpr int OFF_BARS = OFF_V + NV * HALF_BYTES;
+  static constexpr int OFF_EP = OFF_V + NV * HALF_BYTES;  // 8 softmax warps x 32 rows x 128 B
+  static constexpr int OFF_BARS = OFF_EP + 8 * 32 * 128;
   static constexpr int SMEM_BYTES = OFF_BARS + 8192;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t REGS_CTRL = 72, REGS_SOFTMAX = 216;  // 128*72 + 256*216 = 384*168
@@ -244,7 +245,8 @@ static_assert(sizeof(D64Bars) <= 8192, "barrier block");
 __global__ void __launch_bounds__(384, 1)
     attn_kernel_d64(const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v,
-                    const __grid_constant__ CUtensorMap map_q, const AttnArgs a) {
+                    const __grid_constant__ CUtensorMap map_q,
+                    const __grid_constant__ CUtensorMap map_qd, const AttnArgs a) {
   using C = D64Cfg;
   constexpr int D = C::D;
   extern __shared__ __align__(1024) uint8_t smem64[];
@@ -295,6 +297,7 @@ __global__ void __launch_bounds__(384, 1)
     prefetch_tensormap(&map_k);
     prefetch_tensormap(&map_v);
     prefetch_tensormap(&map_q);
+    prefetch_tensormap(&map_qd);
   }
   tc_fence_before();
   __syncthreads();
@@ -441,58 +444,54 @@ __global__ void __launch_bounds__(384, 1)
         mbar_wait_bounded(&bars->drain, 0, &no_abort, nullptr, 0, TO / 4);
       }
     } else if (warp == 2) {
-      // ------------------------------------------------------------------ Q row gather
-      // On the TMA unit: each lane gathers rows 4 lane .. 4 lane + 3 of each 128-row half with one
-      // tile::gather4 copy (four 128-byte rows, swizzled by the TMA unit into the layout the MMA
-      // reads); lane 0 posts the item's byte count on q_full first, so the warp never waits for
-      // the data. The routing entries of the next item are read while this one is in flight.
+      // ------------------------------------------------------------------ Q rows
+      // A routed item's query rows were copied in entry order into one dense array (densify), so
+      // they arrive as one or two 128-row tiles on the TMA unit. A
+      // diagonal item's rows (consecutive tokens of one head, H rows apart) are gathered on the
+      // TMA unit: each lane gathers rows 4 lane .. 4 lane + 3 with one tile::gather4 copy (four
+      // 128-byte rows, swizzled into the layout the MMA reads). Lane 0 posts the item's bytes on
+      // q_full first, so the warp never waits for the data.
       bool ok = true;
       uint32_t issued = 0;
-      auto fetch = [&](const Item& it, int (&e)[8]) {
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          const int m = (x >> 2) * kTile + 4 * lane + (x & 3);
-          e[x] = (it.kind == 1 && m < it.rows) ? __ldg(a.entries + it.start + m) : 0;
-        }
-      };
-      Item cur;
-      int ecur[8];
-      ok = __all_sync(0xffffffffu, pop(0, cur));
-      if (ok) fetch(cur, ecur);
-      for (uint32_t lt = 0; ok && cur.kind >= 0; ++lt) {
+      for (uint32_t lt = 0; ok; ++lt) {
+        Item cur;
+        ok = __all_sync(0xffffffffu, pop(lt, cur));
+        if (!ok || cur.kind < 0) break;
         const uint32_t qb = lt % C::QB;
-        Item nxt;
-        ok = __all_sync(0xffffffffu, pop(lt + 1, nxt));
-        if (!ok) break;
-        int enxt[8];
-        fetch(nxt, enxt);
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->q_empty[qb], ((lt / C::QB) & 1) ^ 1,
                                                        abort_flag, err, kDevTimeoutAttn, TO));
         if (!ok) break;
         const bool hasB = cur.rows > kTile;
-        // query row (t * H + h) of item row m; padding rows repeat a valid row (their results are
-        // never written)
-        int y[8];
+        uint8_t* dst = sQ + qb * C::Q_BYTES;
+        if (cur.kind == 1) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&bars->q_full[qb], (hasB ? 2 : 1) * C::HALF_BYTES);
+            tma_load_2d(dst, &map_qd, &bars->q_full[qb], 0, cur.start);
+            if (hasB)
+              tma_load_2d(dst + C::HALF_BYTES, &map_qd, &bars->q_full[qb], 0, cur.start + kTile);
+          }
+        } else {
+          // query row (t * H + h) of item row m; padding rows repeat a valid row (their results
+          // are never written)
+          int y[8];
 #pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          const int m = (x >> 2) * kTile + 4 * lane + (x & 3);
-          y[x] = (cur.kind == 1) ? a.T0 * a.H + ecur[x] / a.topk
-                                 : (cur.qtok0 + (m < cur.rows ? m : 0)) * a.H + cur.h;
+          for (int x = 0; x < 8; ++x) {
+            const int m = (x >> 2) * kTile + 4 * lane + (x & 3);
+            y[x] = (cur.qtok0 + (m < cur.rows ? m : 0)) * a.H + cur.h;
+          }
+          if (lane == 0)
+            mbar_arrive_expect_tx(&bars->q_full[qb], (hasB ? 2 : 1) * C::HALF_BYTES);
+          __syncwarp();
+          tma_gather4(dst + lane * 512, &map_q, &bars->q_full[qb], 0, y[0], y[1], y[2], y[3]);
+          if (hasB)
+            tma_gather4(dst + C::HALF_BYTES + lane * 512, &map_q, &bars->q_full[qb], 0, y[4],
+                        y[5], y[6], y[7]);
         }
-        if (lane == 0)
-          mbar_arrive_expect_tx(&bars->q_full[qb], (hasB ? 2 : 1) * C::HALF_BYTES);
         __syncwarp();
-        uint8_t* dst = sQ + qb * C::Q_BYTES + lane * 512;
-        tma_gather4(dst, &map_q, &bars->q_full[qb], 0, y[0], y[1], y[2], y[3]);
-        if (hasB)
-          tma_gather4(dst + C::HALF_BYTES, &map_q, &bars->q_full[qb], 0, y[4], y[5], y[6], y[7]);
         ++issued;
-        cur = nxt;
-#pragma unroll
-        for (int x = 0; x < 8; ++x) ecur[x] = enxt[x];
       }
       if (!ok) {
-        // after an abort, let the gathers still in flight land before the CTA exits (bounded)
+        // after an abort, let the loads still in flight land before the CTA exits (bounded)
         volatile int no_abort = 0;
         for (uint32_t x = 0; x < static_cast<uint32_t>(C::QB) && x < issued; ++x) {
           const uint32_t l = issued - 1 - x;
@@ -525,9 +524,11 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const uint32_t t_o = tmem + lane_off + C::tm_o(half, ob);
       const int prev_prow = bars->ep_row[q];
-      const bool prev_valid = prev_prow >= 0;
       const float inv = bars->ep_inv[q];
-      uint4* dst = reinterpret_cast<uint4*>(a.part_o + static_cast<size_t>(prev_prow) * D);
+      // the warp's 32 output rows go through shared memory (16-byte chunk c of row r at chunk
+      // c ^ (r % 8), conflict-free both ways) and leave as whole 128-byte rows, four rows per warp
+      // instruction, instead of 32 scattered 16-byte pieces per instruction
+      uint8_t* ep = smem64 + C::OFF_EP + (warp - 4) * (32 * 128);
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t orr[32];
@@ -535,18 +536,27 @@ __global__ void __launch_bounds__(384, 1)
         tmem_wait_ld();
 #pragma unroll
         for (int x = 0; x < 32; ++x) reg_fence(orr[x]);
-        if (prev_valid) {
 #pragma unroll
-          for (int x = 0; x < 4; ++x)
-            st_part(dst + c0 / 8 + x, make_uint4(
-                pack_bf16x2(__uint_as_float(orr[8 * x + 0]) * inv, __uint_as_float(orr[8 * x + 1]) * inv),
-                pack_bf16x2(__uint_as_float(orr[8 * x + 2]) * inv, __uint_as_float(orr[8 * x + 3]) * inv),
-                pack_bf16x2(__uint_as_float(orr[8 * x + 4]) * inv, __uint_as_float(orr[8 * x + 5]) * inv),
-                pack_bf16x2(__uint_as_float(orr[8 * x + 6]) * inv, __uint_as_float(orr[8 * x + 7]) * inv)));
-        }
+        for (int x = 0; x < 4; ++x)
+          *reinterpret_cast<uint4*>(ep + lane * 128 + (((c0 / 8 + x) ^ (lane & 7)) * 16)) = make_uint4(
+              pack_bf16x2(__uint_as_float(orr[8 * x + 0]) * inv, __uint_as_float(orr[8 * x + 1]) * inv),
+              pack_bf16x2(__uint_as_float(orr[8 * x + 2]) * inv, __uint_as_float(orr[8 * x + 3]) * inv),
+              pack_bf16x2(__uint_as_float(orr[8 * x + 4]) * inv, __uint_as_float(orr[8 * x + 5]) * inv),
+              pack_bf16x2(__uint_as_float(orr[8 * x + 6]) * inv, __uint_as_float(orr[8 * x + 7]) * inv));
       }
       tc_fence_before();
-      if (prev_valid) a.part_lse[prev_prow] = bars->ep_lse[q];
+      __syncwarp();
+      const int c = lane & 7;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = 4 * i + (lane >> 3);
+        const int pr = __shfl_sync(0xffffffffu, prev_prow, r);
+        if (pr >= 0)
+          st_part(reinterpret_cast<uint4*>(a.part_o + static_cast<size_t>(pr) * D) + c,
+                  *reinterpret_cast<const uint4*>(ep + r * 128 + ((c ^ (r & 7)) * 16)));
+      }
+      __syncwarp();
+      if (prev_prow >= 0) a.part_lse[prev_prow] = bars->ep_lse[q];
       return true;
     };
     for (uint32_t lt = 0;; ++lt) {
@@ -1226,11 +1236,27 @@ static bool make_q_rows_map(CUtensorMap* map, const void* base, long long rows, 
              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows, 64] bf16 dense query rows -> 2-D map (64, rows), box (64, 128), 128-byte swizzle, zero
+// fill past the last row.
+static bool make_q_dense_map(CUtensorMap* map, const void* base, long long rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kTile)};
+  cuuint32_t es[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream) {
-  CUtensorMap mk, mv, mq;
+  CUtensorMap mk, mv, mq, mqd;
   if (!make_kv_map(&mk, L.k, L.T, L.G, L.d) || !make_kv_map(&mv, L.v, L.T, L.G, L.d))
     return cudaErrorInvalidValue;
   if (!make_q_rows_map(&mq, L.q, static_cast<long long>(L.T) * L.H, L.d))
+    return cudaErrorInvalidValue;
+  if (L.d == 64 && (!L.qdense || !make_q_dense_map(&mqd, L.qdense, L.qdense_rows)))
     return cudaErrorInvalidValue;
   AttnArgs a;
   a.q = static_cast<const __nv_bfloat16*>(L.q);
@@ -1268,7 +1294,7 @@ cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream) {
     const int smem = D64Cfg::SMEM_BYTES;
     cudaError_t e = cudaFuncSetAttribute(attn_kernel_d64, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_kernel_d64<<<grid, 384, smem, stream>>>(mk, mv, mq, a);
+    attn_kernel_d64<<<grid, 384, smem, stream>>>(mk, mv, mq, mqd, a);
   } else {
     const int smem = PvtCfg::SMEM_BYTES;
     cudaError_t e = cudaFuncSetAttribute(attn_kernel_pvt, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -598,11 +598,13 @@ int gate_stream_schedule(const int32_t* cu_host, int nseq, int H, int G, int d, 
                          int num_ctas, GateSched* S) {
   const int r = H / G, ksel = topk - 1;
   // estimated cost of a tile, in bytes of HBM traffic: every tile writes its rows' selections; a
-  // scored tile also reads its query rows and selects over i past blocks (about one query load's
-  // worth of issue slots at 256 blocks)
+  // scored tile also reads its query rows and selects over i past blocks. The first 32 scores
+  // (one sorted chunk) hide under the query load; each further 64 cost about one more query
+  // load's worth of issue slots (measured at 256 blocks).
   const double q_bytes = 128.0 * d * 2, out_bytes = 128.0 * topk * 4;
   auto tile_cost = [&](int i) -> double {
-    return (ksel > 0 && i > ksel) ? q_bytes + out_bytes + q_bytes * i / 256.0 : out_bytes;
+    return (ksel > 0 && i > ksel) ? q_bytes + out_bytes + q_bytes * std::max(0, i - 32) / 64.0
+                                  : out_bytes;
   };
   double total = 0.0;
   long long n_tiles = 0;

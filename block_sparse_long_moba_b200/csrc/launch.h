@@ -54,6 +54,11 @@ cudaError_t launch_route_scatter(const int32_t* idx, const BlockTables& tb, int 
                                  int topk, int NB, int b0, int nblk, int T0, int max_nb,
                                  int* cursor, int* entries, cudaStream_t stream);
 
+// d = 64: copies the query row of every routed entry of the chunk into qdense (row = entry).
+cudaError_t launch_densify(const int* entries, const int* n_entries, const void* q, int H,
+                           int topk, int T0, long long max_entries, void* qdense, int num_sms,
+                           cudaStream_t stream);
+
 struct AttnLaunch {
   const void* q;
   const void* k;
@@ -61,6 +66,8 @@ struct AttnLaunch {
   const int4* tiles;
   const int* n_routed;
   const int* entries;
+  const void* qdense;      // d = 64: routed query rows, one per entry (nullptr otherwise)
+  long long qdense_rows;   // rows of qdense
   BlockTables tb;
   void* part_o;
   float* part_lse;

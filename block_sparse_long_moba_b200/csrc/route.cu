@@ -14,6 +14,8 @@
 // contiguously. The current block is not routed here: the attention kernel's diagonal tiles
 // cover it. Order inside a bucket is not fixed; results do not depend on it because every
 // attention row is computed independently of the other rows of its tile.
+#include <algorithm>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -188,7 +190,31 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int* __restrict__ coun
     off += c;
     counts[x] = 0;
   }
-  if (tid == nt - 1) *n_tiles = toff;
+  if (tid == nt - 1) {
+    n_tiles[0] = toff;
+    n_tiles[1] = off;  // routed entries of the chunk
+  }
+}
+
+// Densify (d = 64): row p of qdense = the query row of routed entry p, so that the attention
+// kernel reads a work item's gathered rows as dense 128-row tiles. Consecutive entries are written
+// to consecutive rows (coalesced: eight lanes per 128-byte row, four rows per warp instruction);
+// the query rows are read at random and are mostly L2-resident.
+__global__ void __launch_bounds__(256) densify_kernel(const int* __restrict__ entries,
+                                                      const int* __restrict__ n_entries,
+                                                      const __nv_bfloat16* __restrict__ q, int H,
+                                                      int topk, int T0,
+                                                      __nv_bfloat16* __restrict__ qdense) {
+  const int n = *n_entries;
+  const int lane8 = threadIdx.x & 7;
+  const long long stride = static_cast<long long>(gridDim.x) * (blockDim.x >> 3);
+  for (long long p = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 3; p < n;
+       p += stride) {
+    const int e = __ldg(entries + p);
+    const long long row = static_cast<long long>(T0) * H + e / topk;  // t * H + h
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(q + row * 64) + lane8);
+    __stcs(reinterpret_cast<uint4*>(qdense + p * 64) + lane8, v);
+  }
 }
 
 cudaError_t launch_plan(const int32_t* cu_dev, int nseq, int B, int NB, const BlockTables& tb,
@@ -212,6 +238,17 @@ cudaError_t launch_route_count(const int32_t* idx, const BlockTables& tb, int T,
 cudaError_t launch_route_scan(int* counts, int nbk, int* cursor, int4* tiles, int* n_tiles,
                               cudaStream_t stream) {
   route_scan_kernel<<<1, 1024, 0, stream>>>(counts, nbk, cursor, tiles, n_tiles);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_densify(const int* entries, const int* n_entries, const void* q, int H,
+                           int topk, int T0, long long max_entries, void* qdense, int num_sms,
+                           cudaStream_t stream) {
+  const long long want = (max_entries + 31) / 32;  // 32 rows per CTA pass
+  const int grid = static_cast<int>(std::min<long long>(std::max(want, 1LL), 8LL * num_sms));
+  densify_kernel<<<grid, 256, 0, stream>>>(entries, n_entries,
+                                           static_cast<const __nv_bfloat16*>(q), H, topk, T0,
+                                           static_cast<__nv_bfloat16*>(qdense));
   return cudaGetLastError();
 }
 

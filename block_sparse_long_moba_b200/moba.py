@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libmoba.so")
 STATUS = {0: "MOBA_OK", -1: "MOBA_ERR_ARG", -2: "MOBA_ERR_UNSUPPORTED", -3: "MOBA_ERR_WORKSPACE",
           -4: "MOBA_ERR_CUDA", -5: "MOBA_ERR_DEVICE_CHECK", -6: "MOBA_ERR_TIMEOUT"}
 KERNEL_CLASSES = ["centroid", "gate", "route_count", "route_scan", "route_scatter", "attention",
-                  "merge", "plan"]
+                  "merge", "plan", "densify"]
 
 # every symbol include/moba.h declares
 EXPORTS = ["moba_status_string", "moba_version", "moba_workspace_bytes", "moba_centroids",

@@ -154,7 +154,8 @@ int moba_device_status(const void* workspace, void* stream);
  * bracketed by CUDA events recorded on the launching stream. moba_timing_read synchronises the
  * recorded events and writes, for each kernel class, the summed device milliseconds and launch
  * count since the last reset; kernel classes, in order: centroid, gate, route_count, route_scan,
- * route_scatter, attention, merge, plan. Returns the number of classes (8), or a negative status.
+ * route_scatter, attention, merge, plan, densify (d = 64: the routed query rows copied into one
+ * dense array). Returns the number of classes (9), or a negative status.
  */
 int moba_timing_enable(int enable);
 int moba_timing_reset(void);
