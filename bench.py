@@ -427,6 +427,47 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------------- centroid + gate only
+def run_gate_only(args):
+    """Times steps 1-2 alone (moba_centroids + moba_gate_topk through the C ABI, no workspace) on
+    the workload's inputs, one GPU: a small-footprint command for profiling the gate kernels."""
+    from block_sparse_long_moba_b200 import build, moba
+
+    build.build()
+    moba.load_library()
+    torch.cuda.set_device(0)
+    w = wl.WORKLOADS[args.workload]
+    q, k, v, cu = wl.make_inputs(w, seed=0, device="cuda")
+    del v
+    c = moba.moba_centroids(k, cu, w.cu_seqlens, w.block_size)
+    idx = moba.moba_gate_topk(q, c, cu, w.cu_seqlens, w.block_size, w.topk)
+    for _ in range(args.warmup):
+        moba.moba_centroids(k, cu, w.cu_seqlens, w.block_size, out=c)
+        moba.moba_gate_topk(q, c, cu, w.cu_seqlens, w.block_size, w.topk, out=idx)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    cms = gms = 0.0
+    for _ in range(args.steps):
+        ev[0].record()
+        moba.moba_centroids(k, cu, w.cu_seqlens, w.block_size, out=c)
+        ev[1].record()
+        moba.moba_gate_topk(q, c, cu, w.cu_seqlens, w.block_size, w.topk, out=idx)
+        ev[2].record()
+        torch.cuda.synchronize()
+        cms += ev[0].elapsed_time(ev[1])
+        gms += ev[1].elapsed_time(ev[2])
+    cms /= args.steps
+    gms /= args.steps
+    kb = kernel_bytes(w)
+    hbm = read_peaks()["hbm_gbs"]
+    both = (kb["centroid"] + kb["gate"]) / ((cms + gms) / 1e3) / 1e9
+    print(json.dumps({"metric": "centroid + gate GB/s", "value": both, "unit": "GB/s",
+                      "hbm_frac": both / hbm, "workload": w.name, "steps": args.steps,
+                      "centroid_ms": cms, "gate_ms": gms,
+                      "centroid_gbs": kb["centroid"] / (cms / 1e3) / 1e9,
+                      "gate_gbs": kb["gate"] / (gms / 1e3) / 1e9}), flush=True)
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -468,8 +509,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--only", choices=["gate"], default=None,
+                    help="time centroids + gate alone (1 GPU; for profiling)")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.only == "gate":
+        run_gate_only(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
