@@ -68,8 +68,9 @@ int moba_version(void);
 /*
  * Bytes of device workspace moba_attn_fwd needs for this problem (0 on invalid arguments).
  * Depends only on the host-side sizes. The workspace holds block tables, centroids, the routing
- * (when the caller passes no block_idx_out), the inverted routing lists and the per-block partial
- * outputs of one query chunk; chunks are sized so the partials stay under a fixed budget.
+ * (when the caller passes no block_idx_out), the inverted routing lists (at d = 64 with a copy of
+ * each routed query row) and the per-block partial outputs of one query chunk; chunks are sized
+ * so that these per-chunk parts stay under a fixed budget.
  */
 size_t moba_workspace_bytes(int nseq, const int32_t* cu_seqlens_host, int Hq, int Hkv, int d,
                             int block_size, int topk);
