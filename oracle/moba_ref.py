@@ -4,7 +4,8 @@ TEST INFRASTRUCTURE ONLY. Nothing on the product path may import this module: on
 __graft_entry__.smoke() and bench.py's CPU-baseline / reference legs use it. It shares no code
 with the CUDA path (no kernels, headers, helpers or table generators) and is slow on purpose.
 
-What it computes, in the order the method describes it:
+What it computes, in the order the method describes it (plus, for the trainable layer, the
+gradients of step 4 with the routing held fixed: attention_backward):
   1. Keys are cut into fixed-size blocks per sequence; blocks never cross cu_seqlens
      [MoBA README (rpkg.in mirror), "Introducing MoBA": the context is divided into blocks].
   2. Each block is represented by the mean of its keys, per kv head
@@ -234,6 +235,58 @@ def forward(q, k, v, cu_seqlens, block_size, topk, scale, tokens=None):
     rt = select_blocks(q, cents, cu_seqlens, block_size, topk, tokens)
     out, lse = attention(q, k, v, cu_seqlens, block_size, rt.idx, scale, rt.tokens)
     return rt, out, lse
+
+
+def attention_backward(q, k, v, cu_seqlens, block_size, idx_full, scale, d_out) -> tuple:
+    """Gradients of the routed attention with the routing held fixed: dQ [T,H,d], dK, dV [T,G,d].
+
+    MoBA is trained end to end through its block-sparse attention [MoBA README, "Introducing
+    MoBA": trainable block sparse attention]; the top-k gate itself is piecewise constant in q and
+    the centroids, so no gradient flows through the selection (the reading of SURVEY row f1,
+    listed in the design doc). For every row (t, h) over its attended keys u (the keys of its selected
+    blocks, causal inside its own block), with z_u = scale q.k_u, p_u = exp(z_u - LSE) and
+    o = sum_u p_u v_u:
+      dV[u] += p_u dO;  dP_u = dO . v_u;  D = dO . o;  dS_u = p_u (dP_u - D);
+      dQ += scale sum_u dS_u k_u;  dK[u] += scale dS_u q.
+    Keys and values of kv head g collect the terms of all query heads of its group. idx_full:
+    [H, T, topk] local block ids per (head, token), -1 padded; d_out: [T, H, d]. All fp64.
+    """
+    qf, kf, vf, go = to_f64(q), to_f64(k), to_f64(v), to_f64(d_out)
+    T, H, d = qf.shape
+    G = kf.shape[1]
+    r = H // G
+    tokens = np.arange(T, dtype=np.int64)
+    out, lse = attention(q, k, v, cu_seqlens, block_size, idx_full, scale, tokens)  # [T,H,d], [H,T]
+    Dsum = np.einsum("thd,thd->ht", go, out)                                          # [H, T]
+    dq = np.zeros_like(qf)
+    dk = np.zeros_like(kf)
+    dv = np.zeros_like(vf)
+    bt = block_table(cu_seqlens, block_size)
+    s_of, _ = token_position(cu_seqlens, block_size, tokens)
+    sel = np.asarray(idx_full)
+    for b in range(bt.num_blocks):
+        s, j = int(bt.seq[b]), int(bt.local[b])
+        member = (sel == j).any(axis=2) & (s_of == s)[None, :]  # [H, T]
+        if not member.any():
+            continue
+        st, en = int(bt.start[b]), int(bt.end[b])
+        kpos = np.arange(st, en)
+        for g in range(G):
+            hh, tt = np.nonzero(member[g * r:(g + 1) * r])
+            if hh.size == 0:
+                continue
+            hh = hh + g * r
+            kb, vb = kf[st:en, g, :], vf[st:en, g, :]
+            z = scale * (qf[tt, hh, :] @ kb.T)                      # [rows, len]
+            z = np.where(kpos[None, :] <= tt[:, None], z, -np.inf)
+            p = np.exp(z - lse[hh, tt][:, None])
+            dov = go[tt, hh, :]                                     # [rows, d]
+            dv[st:en, g, :] += p.T @ dov
+            dp = dov @ vb.T
+            ds = p * (dp - Dsum[hh, tt][:, None])
+            np.add.at(dq, (tt, hh), scale * (ds @ kb))
+            dk[st:en, g, :] += scale * (ds.T @ qf[tt, hh, :])
+    return dq, dk, dv
 
 
 # ---------------------------------------------------------------------------------------------
