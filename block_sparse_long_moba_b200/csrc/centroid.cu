@@ -54,18 +54,13 @@ __global__ void __launch_bounds__(256) centroid_kernel(const __nv_bfloat16* __re
     }
   };
   int t = lo + rr;
-  for (; t + 3 * RP < hi; t += 4 * RP) {
-    const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(src + static_cast<size_t>(t) * row_stride));
-    const uint4 v1 =
-        __ldg(reinterpret_cast<const uint4*>(src + static_cast<size_t>(t + RP) * row_stride));
-    const uint4 v2 =
-        __ldg(reinterpret_cast<const uint4*>(src + static_cast<size_t>(t + 2 * RP) * row_stride));
-    const uint4 v3 =
-        __ldg(reinterpret_cast<const uint4*>(src + static_cast<size_t>(t + 3 * RP) * row_stride));
-    add(v0);
-    add(v1);
-    add(v2);
-    add(v3);
+  for (; t + 7 * RP < hi; t += 8 * RP) {  // eight rows in flight per thread
+    uint4 v[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x)
+      v[x] = __ldg(reinterpret_cast<const uint4*>(src + static_cast<size_t>(t + x * RP) * row_stride));
+#pragma unroll
+    for (int x = 0; x < 8; ++x) add(v[x]);
   }
   for (; t < hi; t += RP)
     add(__ldg(reinterpret_cast<const uint4*>(src + static_cast<size_t>(t) * row_stride)));

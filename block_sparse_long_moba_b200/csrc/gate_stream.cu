@@ -102,6 +102,48 @@ __device__ __forceinline__ void bitonic32_desc(uint32_t (&k)[32]) {
   }
 }
 
+// Bitonic sorting network over N (a power of two) keys, descending (static indices only).
+template <int N>
+__device__ __forceinline__ void bitonic_desc(uint32_t (&k)[N]) {
+#pragma unroll
+  for (int size = 2; size <= N; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int a = 0; a < N; ++a) {
+        const int b = a ^ stride;
+        if (b > a) {
+          const uint32_t hi = max(k[a], k[b]), lo = min(k[a], k[b]);
+          if ((a & size) == 0 || size == N) {
+            k[a] = hi;
+            k[b] = lo;
+          } else {
+            k[a] = lo;
+            k[b] = hi;
+          }
+        }
+      }
+    }
+  }
+}
+
+// Sorts a bitonic sequence of N keys descending (the merge stages of the network).
+template <int N>
+__device__ __forceinline__ void bitonic_clean_desc(uint32_t (&k)[N]) {
+#pragma unroll
+  for (int stride = N >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+    for (int a = 0; a < N; ++a) {
+      const int b = a ^ stride;
+      if (b > a) {
+        const uint32_t hi = max(k[a], k[b]), lo = min(k[a], k[b]);
+        k[a] = hi;
+        k[b] = lo;
+      }
+    }
+  }
+}
+
 // Bitonic sorting network over N (a power of two) int registers, ascending.
 template <int N>
 __device__ __forceinline__ void bitonic_asc(int (&k)[N]) {
@@ -486,9 +528,30 @@ __global__ void __launch_bounds__(384, 1)
         for (int x = 0; x < 32; ++x) reg_fence(sr[x]);
 #pragma unroll
         for (int x = 0; x < 32; ++x) sr[x] = (x < n) ? gs_key(__uint_as_float(sr[x]), x) : 0u;
-        bitonic32_desc(sr);
+        if (KCAP <= 16) {
+          // the 16 best of 32: both halves sorted, the larger of a[x] and b[15 - x] (a bitonic
+          // sequence holding the 16 largest keys) sorted again; a row of at most 16 columns
+          // only needs its first half sorted
+          uint32_t ha[16], hb[16];
 #pragma unroll
-        for (int x = 0; x < KCAP; ++x) kk[x] = sr[x];
+          for (int x = 0; x < 16; ++x) {
+            ha[x] = sr[x];
+            hb[x] = sr[16 + x];
+          }
+          bitonic_desc<16>(ha);
+          if (n > 16) {
+            bitonic_desc<16>(hb);
+#pragma unroll
+            for (int x = 0; x < 16; ++x) ha[x] = max(ha[x], hb[15 - x]);
+            bitonic_clean_desc<16>(ha);
+          }
+#pragma unroll
+          for (int x = 0; x < KCAP; ++x) kk[x] = ha[x];
+        } else {
+          bitonic32_desc(sr);
+#pragma unroll
+          for (int x = 0; x < KCAP; ++x) kk[x] = sr[x];
+        }
       }
       for (int cc = 32; cc < n; cc += 32) {
         uint32_t sr[32];
