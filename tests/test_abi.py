@@ -92,3 +92,13 @@ def test_centroids_and_gate_host_side_errors(lib):
     assert lib.moba_gate_topk(FAKE, FAKE, FAKE, cu, 1, 2, 2, 64, 128, 0, FAKE, None) == -1
     assert lib.moba_gate_topk(FAKE, None, FAKE, cu, 1, 2, 2, 64, 128, 3, FAKE, None) == -1
     assert lib.moba_gate_topk(FAKE, FAKE, FAKE, _cu([0, 0]), 1, 2, 2, 64, 128, 3, FAKE, None) == 0
+
+
+def test_timing_classes_match_the_binding(lib):
+    """moba_timing_read reports one entry per kernel class, in the binding's order (no GPU: with
+    timing off nothing is recorded and no event is touched)."""
+    from block_sparse_long_moba_b200 import moba
+    assert lib.moba_timing_reset() == 0
+    n = lib.moba_timing_read(None, None, 0)
+    assert n == len(moba.KERNEL_CLASSES) == 9
+    assert moba.KERNEL_CLASSES[-1] == "densify"

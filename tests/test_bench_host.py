@@ -91,3 +91,20 @@ def test_attention_traffic_only_for_the_sources_it_was_taken_on(tmp_path, monkey
     assert bench.attention_traffic("w") == 123.0
     (csrc / "attn.cu").write_text("// changed")  # the kernel changed since the capture
     assert bench.attention_traffic("w") is None
+
+
+def test_kernel_bytes_count_densify_at_d64_only():
+    import bench
+    from block_sparse_long_moba_b200 import workloads as wl
+    small = bench.kernel_bytes(wl.WORKLOADS["routing_64k_b128"])
+    big = bench.kernel_bytes(wl.WORKLOADS["llama8b_128k"])
+    assert "densify" in small and "densify" not in big
+    # every routed entry: its 4-byte entry read, its 128-byte query row read and written
+    w = wl.WORKLOADS["routing_64k_b128"]
+    entries = 0  # routed (t, h, slot): every selected past block of every row
+    for s in range(w.nseq):
+        L = w.cu_seqlens[s + 1] - w.cu_seqlens[s]
+        for i in range((L + w.block_size - 1) // w.block_size):
+            entries += min(w.block_size, L - i * w.block_size) * (min(w.topk, i + 1) - 1)
+    entries *= w.hq
+    assert entries > 0 and small["densify"] == entries * (4 + 4 * w.d)
