@@ -4,9 +4,12 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/moba.h"
 #include "common.cuh"
@@ -25,9 +28,15 @@ enum KernelClass {
 std::atomic<long long> g_launches{0};
 
 // ------------------------------------------------------------------------------- timing hooks
+// Timing starts enabled when the process sets MOBA_TIMING=1.
+bool timing_from_env() {
+  const char* v = std::getenv("MOBA_TIMING");
+  return v && v[0] == '1' && v[1] == '\0';
+}
+
 struct Timing {
   std::mutex mu;
-  bool enabled = false;
+  bool enabled = timing_from_env();
   double ms[kNumClasses] = {0};
   long long n[kNumClasses] = {0};
   struct Pending { int cls; cudaEvent_t a, b; };
@@ -42,14 +51,23 @@ struct Timing {
 };
 Timing& timing() { static Timing t; return t; }
 
-struct Scope {  // brackets one kernel launch with events when timing is enabled
+const char* const kClassNames[kNumClasses] = {"moba_centroids", "moba_gate", "moba_route_count",
+                                               "moba_route_scan", "moba_route_scatter",
+                                               "moba_attention", "moba_merge", "moba_plan",
+                                               "moba_densify"};
+
+// Brackets one kernel launch: an NVTX range named for its class (seen by profilers; a no-op
+// otherwise) and, when timing is enabled, CUDA events on the launching stream.
+struct Scope {
   int cls; cudaStream_t s; cudaEvent_t a = nullptr, b = nullptr; bool on = false;
   Scope(int c, cudaStream_t st) : cls(c), s(st) {
+    nvtxRangePushA(kClassNames[c]);
     Timing& T = timing();
     std::lock_guard<std::mutex> g(T.mu);
     if (T.enabled) { on = true; a = T.get(); b = T.get(); cudaEventRecord(a, s); }
   }
   void done() {
+    nvtxRangePop();
     g_launches.fetch_add(1);
     if (!on) return;
     cudaEventRecord(b, s);
@@ -406,8 +424,9 @@ int moba_device_status(const void* workspace, void* stream) {
 int moba_timing_enable(int enable) {
   Timing& T = timing();
   std::lock_guard<std::mutex> g(T.mu);
+  const int was = T.enabled ? 1 : 0;
   T.enabled = enable != 0;
-  return MOBA_OK;
+  return was;
 }
 
 int moba_timing_reset(void) {

@@ -151,8 +151,12 @@ int moba_attn_fwd_noalloc(const void* q, const void* k, const void* v,
 int moba_device_status(const void* workspace, void* stream);
 
 /*
- * Instrumentation (off by default). When enabled, every kernel launch of the library is
- * bracketed by CUDA events recorded on the launching stream. moba_timing_read synchronises the
+ * Instrumentation (off by default; on from the start when the environment sets MOBA_TIMING=1).
+ * When enabled, every kernel launch of the library is bracketed by CUDA events recorded on the
+ * launching stream. Every launch is also bracketed by an NVTX range named for its class
+ * (moba_centroids, moba_gate, ...), which profilers show and which costs nothing without one.
+ * moba_timing_enable switches the timing on (enable != 0) or off and returns whether it was on
+ * before the call (1 or 0). moba_timing_read synchronises the
  * recorded events and writes, for each kernel class, the summed device milliseconds and launch
  * count since the last reset; kernel classes, in order: centroid, gate, route_count, route_scan,
  * route_scatter, attention, merge, plan, densify (d = 64: the routed query rows copied into one

@@ -102,3 +102,23 @@ def test_timing_classes_match_the_binding(lib):
     n = lib.moba_timing_read(None, None, 0)
     assert n == len(moba.KERNEL_CLASSES) == 9
     assert moba.KERNEL_CLASSES[-1] == "densify"
+
+
+@pytest.mark.parametrize("value,was_on", [("1", "1"), ("0", "0"), (None, "0")])
+def test_timing_can_start_from_the_environment(value, was_on):
+    """MOBA_TIMING=1 turns the timing hooks on when the library loads: in a fresh process,
+    moba_timing_enable(0) then reports that timing was on (no GPU is touched)."""
+    import subprocess
+    import sys
+    code = ("import sys; sys.path.insert(0, %r)\n"
+            "from block_sparse_long_moba_b200 import moba\n"
+            "lib = moba.load_library()\n"
+            "print(lib.moba_timing_enable(0), lib.moba_timing_enable(0))\n") % ROOT
+    env = dict(os.environ)
+    env.pop("MOBA_TIMING", None)
+    if value is not None:
+        env["MOBA_TIMING"] = value
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env,
+                         timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert out.stdout.split() == [was_on, "0"]
