@@ -213,14 +213,24 @@ def oracle_sample_rate(w: wl.Workload, q, k, v, target_s: float = 15.0, seed: in
 ATTN_SOURCES = ("attn.cu", "sm100.cuh", "common.cuh")
 
 
+def _code_only(text: str) -> str:
+    """C++ source without its comments and with whitespace collapsed: what the compiler sees, so
+    that editing a comment does not orphan a profile taken on the same code."""
+    import re
+
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def attention_source_hash() -> str:
-    """sha256 over the attention kernel's source files, in a fixed order."""
+    """sha256 over the code (comments removed) of the attention kernel's sources, fixed order."""
     import hashlib
 
     h = hashlib.sha256()
     for name in ATTN_SOURCES:
-        with open(os.path.join(ROOT, "block_sparse_long_moba_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "block_sparse_long_moba_b200", "csrc", name)) as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()
 
 

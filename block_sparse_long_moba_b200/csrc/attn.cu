@@ -23,10 +23,11 @@
 // S_x(j), the arrival of S_x(j) implies O_x is complete, so a rescale never waits.
 //
 // Warp roles (384 threads): warp 0 = TMA producer of K/V sub-tiles; warp 1 = TMEM owner and MMA
-// issuer (both run converged and let elect.sync pick the issuing lane); warps 2-3 = Q row gather (cp.async into the swizzled layout); warps 4-7 = softmax and
-// epilogue of half A; warps 8-11 = the same for half B. Every wait is bounded (2 s); on a timeout
-// the kernel raises a CTA abort flag, records a status code, drains what it has in flight and
-// returns.
+// issuer (both run converged and let elect.sync pick the issuing lane); warps 2-3 = query rows
+// (d = 128: gathered by the TMA unit and by cp.async in parallel; d = 64: see its kernel);
+// warps 4-7 = softmax and epilogue of half A; warps 8-11 = the same for half B. Every wait is
+// bounded (2 s); on a timeout the kernel raises a CTA abort flag, records a status code, drains
+// what it has in flight and returns.
 #include "common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
@@ -195,15 +196,17 @@ __device__ __forceinline__ bool ring_consume(ItemRing* ring, uint32_t lt, Item& 
 // d = 64 kernel.
 //
 // Roles (384 threads): warp 0 = TMA producer of K/V sub-tiles; warp 1 = TMEM owner and MMA issuer
-// (the whole warp runs converged, elect.sync picks the issuing lane); warp 2 = Q row gather;
-// warp 3 = item scheduler; warps 4-7 = softmax and epilogue of half A; warps 8-11 = half B.
+// (the whole warp runs converged, elect.sync picks the issuing lane); warp 2 = query rows (TMA
+// tile loads from the densified rows, or a tile::gather4 gather for diagonal items); warp 3 =
+// item scheduler; warps 4-7 = softmax and epilogue of half A; warps 8-11 = half B.
 //
 // Small blocks make small items (a 128-key block is one sub-tile), so the per-item overheads are
 // what this kernel is shaped around:
-//   * the gather first reads the item's routing entries with coalesced loads, then issues its
-//     16-byte row copies and keeps two items in flight (cp.async groups), QB items ahead;
+//   * a routed item's query rows were densified in list order beforehand, so they arrive as one
+//     or two 128-row TMA tiles, QB items ahead;
 //   * O accumulators are double-buffered in TMEM per half (item parity), and the epilogue of an
-//     item runs after the next item's softmax, so it never delays the tensor pipe;
+//     item runs after the next item's softmax, so it never delays the tensor pipe; it writes
+//     whole 128-byte rows through a per-warp staging area in shared memory;
 //   * an item of at most 128 rows (every diagonal item of a 128-key block, the tail item of a
 //     routed list) runs on half A only: half B issues no MMA and its warps skip the item.
 struct D64Cfg {

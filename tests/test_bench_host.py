@@ -80,8 +80,11 @@ def test_attention_traffic_only_for_the_sources_it_was_taken_on(tmp_path, monkey
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     csrc = tmp_path / "block_sparse_long_moba_b200" / "csrc"
     csrc.mkdir(parents=True)
+    def code(name):
+        return "int v_%s;" % name.replace(".", "_")
+
     for name in bench.ATTN_SOURCES:
-        (csrc / name).write_text("// " + name)
+        (csrc / name).write_text(code(name) + "  // " + name)
     (tmp_path / "profiles").mkdir()
     rec = tmp_path / "profiles" / "attention_w_traffic.json"
     assert bench.attention_traffic("w") is None  # no record
@@ -89,7 +92,9 @@ def test_attention_traffic_only_for_the_sources_it_was_taken_on(tmp_path, monkey
     rec.write_text(json.dumps({"bytes_per_launch": 123.0,
                                "kernel_sources_sha256": bench.attention_source_hash()}))
     assert bench.attention_traffic("w") == 123.0
-    (csrc / "attn.cu").write_text("// changed")  # the kernel changed since the capture
+    (csrc / "attn.cu").write_text(code("attn.cu") + "  /* a comment edit */ // keeps the record")
+    assert bench.attention_traffic("w") == 123.0
+    (csrc / "attn.cu").write_text("int y;  // changed code")  # the kernel changed
     assert bench.attention_traffic("w") is None
 
 
