@@ -96,6 +96,56 @@ def kernel_bytes(w: wl.Workload) -> dict:
     }
 
 
+def executed_flops(w: wl.Workload, idx: torch.Tensor) -> float:
+    """Tile FLOPs the attention kernel issues for one step, from the routing it was given.
+
+    Work items are 256 query rows (two 128-row halves) against every 128-key sub-tile of one
+    block: a routed item covers up to 256 rows of one (kv head, past block) list, a diagonal item
+    up to 256 consecutive tokens of one head inside its own block against the keys up to its last
+    query. At d = 128 both halves always run (the value product is issued for 256 rows at once);
+    at d = 64 an item of at most 128 rows runs on one half. Each 128 x 128 sub-tile pair costs
+    4 d 128^2 FLOPs (QK^T and PV). Routed-list lengths are counted from idx on the device."""
+    T, H, G, d, B, k = w.total_tokens, w.hq, w.hkv, w.d, w.block_size, w.topk
+    dev = idx.device
+    r = H // G
+    bot = wl.block_of_token(w, dev)                         # global block of every token
+    blk_off = [0]
+    for nb in w.seq_blocks():
+        blk_off.append(blk_off[-1] + nb)
+    seq_of_blk = torch.repeat_interleave(torch.arange(w.nseq, device=dev),
+                                         torch.tensor(w.seq_blocks(), device=dev))
+    base = torch.tensor(blk_off[:-1], device=dev, dtype=torch.int64)[seq_of_blk[bot]]
+    i_tok = (bot - base)[:, None]                           # local block of every token
+    NB = w.num_blocks
+    counts = torch.zeros(G * NB, dtype=torch.int64, device=dev)
+    for h in range(H):
+        j = idx[h].to(torch.int64)
+        ok = (j >= 0) & (j < i_tok)
+        b = (base[:, None] + j)[ok]
+        counts[(h // r) * NB:(h // r + 1) * NB] += torch.bincount(b, minlength=NB)
+    blk_len = []
+    for s in range(w.nseq):
+        L = w.cu_seqlens[s + 1] - w.cu_seqlens[s]
+        blk_len += [min(B, L - x * B) for x in range((L + B - 1) // B)]
+    nsub = torch.tensor([(n + 127) // 128 for n in blk_len], device=dev, dtype=torch.int64)
+    nsub_g = nsub.repeat(G)
+    full = counts // 256
+    tail = counts % 256
+    if d == 128:
+        rows_tail = torch.where(tail > 0, 256, 0)
+    else:
+        rows_tail = torch.where(tail > 128, 256, torch.where(tail > 0, 128, 0))
+    routed_rows_x_sub = int(((full * 256 + rows_tail) * nsub_g).sum().item())
+    diag = 0
+    for n in blk_len:
+        for q0 in range(0, n, 256):
+            rows = min(256, n - q0)
+            exec_rows = 256 if (d == 128 or rows > 128) else 128
+            diag += exec_rows * ((q0 + rows + 127) // 128)
+    diag *= H
+    return 4.0 * d * 128 * (routed_rows_x_sub + diag)
+
+
 def job_throughput(world: int, tokens_per_rank: int, ms_step_max: float) -> float:
     """Whole-job query tokens/s: every rank processes its own problem (weak scaling), timed as
     the max over ranks."""
@@ -181,32 +231,59 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
-def oracle_sample_rate(w: wl.Workload, q, k, v, target_s: float = 15.0, seed: int = 0) -> dict:
-    """Time the fp64 oracle (as it stands) on a bounded sample of query tokens (all heads):
-    centroids of the whole K (charged pro rata to the sample), gate and attention of the sample.
-    Returns query-tokens/s."""
-    from oracle import moba_ref as ref
+def oracle_target_seconds(args) -> float:
+    """Seconds of oracle work per sample, the same for the reference arm's steps and the
+    CPU-baseline leg (so both time the same sample size): at most --cpu-seconds, and small
+    enough that --steps + --warmup samples take about four minutes."""
+    return max(1.0, min(args.cpu_seconds, 240.0 / max(args.steps + args.warmup, 1)))
 
-    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
-    t0 = time.perf_counter()
-    cents = ref.centroids(kc, w.cu_seqlens, w.block_size)
-    t_cent = time.perf_counter() - t0
-    rng = np.random.default_rng(seed)
-    T = w.total_tokens
-    done_tok, t_rows, n = 0, 0.0, 4
-    while t_rows < target_s and done_tok < T:
-        toks = np.sort(rng.choice(T, size=min(n, T), replace=False))
+
+class OracleSampler:
+    """Times the fp64 oracle (as it stands) on bounded samples of one workload's query tokens.
+
+    One sample = one oracle call (gate + attention) on n seeded random query tokens, all heads,
+    plus the centroids of the whole K, computed once and charged pro rata (n / T of its time).
+    An oracle call has a fixed cost (it walks every block of K and V once) besides its per-token
+    cost, so its rate depends on n: the sample size is fixed once, from an untimed calibration
+    call on 64 tokens, so that one sample takes about `target_s`, and every timed sample (of the
+    reference arm and of the CPU-baseline leg alike) uses that same n."""
+
+    def __init__(self, w: wl.Workload, q, k, v, target_s: float, seed: int = 0):
+        from oracle import moba_ref as ref
+
+        self.ref, self.w = ref, w
+        self.qc, self.kc, self.vc = q.cpu(), k.cpu(), v.cpu()
+        t0 = time.perf_counter()
+        self.cents = ref.centroids(self.kc, w.cu_seqlens, w.block_size)
+        self.t_cent = time.perf_counter() - t0
+        self.rng = np.random.default_rng(seed)
+        T = w.total_tokens
+        n0 = min(64, T)
+        t_cal = self._call(n0)
+        self.n = int(min(T, 4096, max(n0, round(n0 * target_s / max(t_cal, 1e-6)))))
+
+    def _call(self, n: int) -> float:
+        T = self.w.total_tokens
+        toks = np.sort(self.rng.choice(T, size=min(n, T), replace=False))
         t1 = time.perf_counter()
-        rt = ref.select_blocks(qc, cents, w.cu_seqlens, w.block_size, w.topk, toks)
-        ref.attention(qc, kc, vc, w.cu_seqlens, w.block_size, rt.idx, w.scale, toks)
-        t_rows += time.perf_counter() - t1
-        done_tok += len(toks)
-        n = min(n * 2, 4096)
-    charged = t_rows + t_cent * done_tok / T
-    return {"value": done_tok / charged, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{done_tok} random query tokens x all {w.hq} heads of {w.name} "
-                      f"(gate + attention {t_rows:.1f} s) + centroids of all {w.num_blocks} blocks "
-                      f"({t_cent:.1f} s, charged pro rata {done_tok}/{T})"}
+        rt = self.ref.select_blocks(self.qc, self.cents, self.w.cu_seqlens, self.w.block_size,
+                                    self.w.topk, toks)
+        self.ref.attention(self.qc, self.kc, self.vc, self.w.cu_seqlens, self.w.block_size,
+                           rt.idx, self.w.scale, toks)
+        return time.perf_counter() - t1
+
+    def sample(self) -> dict:
+        """One timed sample; returns its rate in query-tokens/s and what it covered."""
+        t_rows = self._call(self.n)
+        T = self.w.total_tokens
+        charged = t_rows + self.t_cent * self.n / T
+        w = self.w
+        return {"value": self.n / charged, "unit": UNIT, "cores": blas_threads(),
+                "kind": "oracle", "seconds": charged,
+                "sample": f"{self.n} random query tokens x all {w.hq} heads of {w.name} per "
+                          f"sample (gate + attention {t_rows:.1f} s) + centroids of all "
+                          f"{w.num_blocks} blocks ({self.t_cent:.1f} s, charged pro rata "
+                          f"{self.n}/{T})"}
 
 
 # ---------------------------------------------------------------------------------- traffic
@@ -292,17 +369,20 @@ def physical_gpu_index(local: int) -> int:
 
 
 # ----------------------------------------------------------------------------------- our arm
-def run_ours(args):
-    from block_sparse_long_moba_b200 import build, moba
+# Workloads timed beside the headline one (one GPU only): the 1M-token shape the metric is also
+# quoted on and the two small-block shapes, each on its own buffers (freed before the next).
+EXTRA_WORKLOADS = (("llama8b_1m", 3), ("routing_64k_b128", 10), ("varlen_512k_b128", 10))
 
-    world, rank, local = dist_setup(args.gpus)
-    if rank == 0:
-        build.build()
-    barrier(world)
-    moba.load_library()
-    w = wl.WORKLOADS[args.workload]
+
+def measure(w: wl.Workload, steps: int, warmup: int, world: int, rank: int, local: int,
+            seed: int, e2e: bool, clocks_on: bool) -> dict:
+    """Times `steps` forward passes of `w` (inputs resident in HBM), bracketed by a barrier and a
+    device synchronisation on both sides, max over ranks; optionally the end-to-end variant with
+    pinned host buffers copied in and out every step. Returns the raw figures of this rank."""
+    from block_sparse_long_moba_b200 import moba
+
     dev = torch.device("cuda", torch.cuda.current_device())
-    q, k, v, cu = wl.make_inputs(w, seed=rank, device=dev)
+    q, k, v, cu = wl.make_inputs(w, seed=seed, device=dev)
     T, H, d = w.total_tokens, w.hq, w.d
     o = torch.empty_like(q)
     lse = torch.empty((H, T), dtype=torch.float32, device=dev)
@@ -315,17 +395,17 @@ def run_ours(args):
         moba.moba_attn_fwd(q, k, v, cu, w.cu_seqlens, w.block_size, w.topk, w.scale,
                            block_idx_out=idx, o=o, lse=lse, workspace=ws, stream=stream)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     status = moba.moba_device_status(ws)
     if status != 0:
-        raise RuntimeError(f"device status {status} after warm-up")
+        raise RuntimeError(f"{w.name}: device status {status} after warm-up")
 
     # ---- device-timed region: inputs resident in HBM
     moba.timing_reset()
     moba.timing_enable(True)
-    clocks = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
+    clocks = ClockSampler(physical_gpu_index(local)) if (rank == 0 and clocks_on) else None
     if clocks:
         clocks.start()
         time.sleep(0.3)
@@ -334,7 +414,7 @@ def run_ours(args):
     barrier(world)
     torch.cuda.synchronize()
     ev0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         step()
     ev1.record(stream)
     torch.cuda.synchronize()
@@ -347,7 +427,11 @@ def run_ours(args):
     ms = max_over_ranks(ms_local, world)
     status = moba.moba_device_status(ws)
     if status != 0:
-        raise RuntimeError(f"device status {status} after the timed region")
+        raise RuntimeError(f"{w.name}: device status {status} after the timed region")
+    out = {"ms": ms, "ms_local": ms_local, "per_kernel": per_kernel, "launches": launches,
+           "clocks": clk, "executed_flops": executed_flops(w, idx)}
+    if not e2e:
+        return out
 
     # ---- end to end through the public API: pinned host inputs -> device -> host outputs
     qh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True).copy_(q)
@@ -369,7 +453,7 @@ def run_ours(args):
         oh.copy_(o, non_blocking=True)
         lh.copy_(lse, non_blocking=True)
 
-    e2e_steps = max(1, min(args.steps, 5))
+    e2e_steps = max(1, min(steps, 5))
     e2e_step()
     torch.cuda.synchronize()
     barrier(world)
@@ -378,36 +462,101 @@ def run_ours(args):
         e2e_step()
     ev1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world) / e2e_steps
+    out["e2e_ms"] = max_over_ranks(ev0.elapsed_time(ev1), world) / e2e_steps
+    out["h2d"], out["d2h"] = h2d, d2h
+    out["inputs"] = (q, k, v)
+    return out
+
+
+def summarize(w: wl.Workload, m: dict, steps: int, world: int, peaks: dict) -> dict:
+    """Throughput, TFLOP/s (useful and executed), the attention roofline and per-kernel figures
+    of one measured workload."""
+    ms_step = m["ms"] / steps
+    uf, xf = useful_flops(w), m["executed_flops"]
+    per_kernel = m["per_kernel"]
+    attn_ms, attn_n = per_kernel["attention"]
+    attn_step_s = attn_ms / steps / 1e3                   # attention time per step
+    peak = peaks["bf16_tflops_sustained"]
+    achieved = uf / attn_step_s / 1e12
+    kb = kernel_bytes(w)
+    kern = {}
+    for name, (kms, kn) in per_kernel.items():
+        if kn == 0:
+            continue
+        ent = {"ms_per_launch": kms / kn, "launches": kn, "share": kms / max(m["ms_local"], 1e-9)}
+        if name in kb:
+            # kb holds the bytes of one whole step; a chunked problem launches a kernel several
+            # times per step, so divide by the kernel's time per step
+            gbs = kb[name] / (kms / steps / 1e3) / 1e9
+            ent["gbs"] = gbs
+            ent["hbm_frac"] = gbs / peaks["hbm_gbs"]
+        kern[name] = ent
+    if "gate" in kern:
+        kern["gate"]["gate_tflops_fp32"] = gate_flops(w) / (kern["gate"]["ms_per_launch"] / 1e3) / 1e12
+    cg = None
+    if "centroid" in per_kernel and "gate" in per_kernel:
+        cg_s = (per_kernel["centroid"][0] + per_kernel["gate"][0]) / steps / 1e3
+        cg = (kb["centroid"] + kb["gate"]) / cg_s / 1e9 / peaks["hbm_gbs"]
+    return {
+        "ms_per_step": ms_step,
+        "value": job_throughput(world, w.total_tokens, ms_step),
+        "tflops_useful": uf * world / (ms_step / 1e3) / 1e12,
+        "tflops_executed": xf * world / (ms_step / 1e3) / 1e12,
+        "attention": {"achieved_useful": achieved, "achieved_executed": xf / attn_step_s / 1e12,
+                      "frac": achieved / peak, "frac_executed": xf / attn_step_s / 1e12 / peak,
+                      "frac_of_burst": achieved / peaks["bf16_tflops"],
+                      "useful_tflop": uf / 1e12, "executed_tflop": xf / 1e12,
+                      "ms_per_step": attn_ms / steps},
+        "centroid_gate_hbm_frac": cg,
+        "kernels": kern,
+        "launches_per_step": m["launches"] / steps,
+    }
+
+
+def run_ours(args):
+    from block_sparse_long_moba_b200 import build, moba
+
+    world, rank, local = dist_setup(args.gpus)
+    if rank == 0:
+        build.build()
+    barrier(world)
+    moba.load_library()
+    w = wl.WORKLOADS[args.workload]
+    peaks = read_peaks()
+    m = measure(w, args.steps, args.warmup, world, rank, local, seed=rank, e2e=True,
+                clocks_on=True)
+    summ = summarize(w, m, args.steps, world, peaks) if rank == 0 else None
+    T, H, d = w.total_tokens, w.hq, w.d
+    q, k, v = m.pop("inputs")
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sampler = OracleSampler(w, q, k, v, target_s=oracle_target_seconds(args))
+        cpu = sampler.sample()
+    del q, k, v
+    torch.cuda.empty_cache()
+
+    extra = {}
+    if world == 1 and not args.no_extra:
+        for name, steps in EXTRA_WORKLOADS:
+            if name == w.name:
+                continue
+            wx = wl.WORKLOADS[name]
+            mx = measure(wx, steps, 2, world, rank, local, seed=rank, e2e=False, clocks_on=True)
+            sx = summarize(wx, mx, steps, world, peaks)
+            extra[name] = {"steps": steps, "warmup": 2, **sx, "clocks": mx["clocks"],
+                           "config": {"T": wx.total_tokens, "hq": wx.hq, "hkv": wx.hkv,
+                                      "d": wx.d, "block_size": wx.block_size, "topk": wx.topk,
+                                      "nseq": wx.nseq}}
+            del mx
+            torch.cuda.empty_cache()
 
     if rank == 0:
-        peaks = read_peaks()
-        ms_step = ms / args.steps
-        value = job_throughput(world, T, ms_step)
-        uf = useful_flops(w)
-        attn_ms, attn_n = per_kernel["attention"]
-        attn_avg = attn_ms / max(attn_n, 1)
-        launches_per_step = max(attn_n // args.steps, 1)
-        achieved = uf / launches_per_step / (attn_avg / 1e3) / 1e12
+        ms_step = summ["ms_per_step"]
+        att = summ["attention"]
         peak = peaks["bf16_tflops_sustained"]
-        kb = kernel_bytes(w)
-        kern = {}
-        for name, (kms, kn) in per_kernel.items():
-            if kn == 0:
-                continue
-            ent = {"ms_per_launch": kms / kn, "launches": kn, "share": kms / max(ms_local, 1e-9)}
-            if name in kb:
-                # kb holds the bytes of one whole step; a chunked problem launches a kernel
-                # several times per step, so divide by the kernel's time per step
-                gbs = kb[name] / (kms / args.steps / 1e3) / 1e9
-                ent["gbs"] = gbs
-                ent["hbm_frac"] = gbs / peaks["hbm_gbs"]
-            kern[name] = ent
-        if "gate" in kern:
-            kern["gate"]["gate_tflops_fp32"] = gate_flops(w) / (kern["gate"]["ms_per_launch"] / 1e3) / 1e12
         traffic = attention_traffic(w.name)
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "metric": METRIC, "value": summ["value"], "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; Q,V ~ N(0,1), K = N(0,1) + per-block offset)",
@@ -415,22 +564,28 @@ def run_ours(args):
                        "block_size": w.block_size, "topk": w.topk, "nseq": w.nseq,
                        "parallelism": f"independent problem per GPU x{world}",
                        "l2": "no flush: Q/K/V inputs are larger than L2"},
-            "tflops_useful": uf * world / (ms_step / 1e3) / 1e12,
-            "tflops_frac_of_peak_sustained": uf / (ms_step / 1e3) / 1e12 / peak,
-            "roofline": {"kernel": "attention", "bound": "tensor", "achieved": achieved,
-                         "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "tflops_useful": summ["tflops_useful"],
+            "tflops_executed": summ["tflops_executed"],
+            "tflops_frac_of_peak_sustained": summ["tflops_useful"] / world / peak,
+            "roofline": {"kernel": "attention", "bound": "tensor", "achieved": att["achieved_useful"],
+                         "peak": peak, "unit": "TFLOP/s", "frac": att["frac"],
                          "peak_kind": f"bf16 dense sustained, {peaks['source']}",
-                         "frac_of_burst": achieved / peaks["bf16_tflops"],
+                         "frac_of_burst": att["frac_of_burst"],
+                         "achieved_executed": att["achieved_executed"],
+                         "frac_executed": att["frac_executed"],
                          "traffic": traffic},
-            "kernels": kern,
-            "gpu_launches": launches,
-            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms},
-            "clocks": clk,
+            "centroid_gate_hbm_frac": summ["centroid_gate_hbm_frac"],
+            "kernels": summ["kernels"],
+            "gpu_launches": m["launches"],
+            "e2e": {"value": world * T / (m["e2e_ms"] / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": m["h2d"], "d2h_bytes_per_step": m["d2h"],
+                    "ms_per_step": m["e2e_ms"]},
+            "clocks": m["clocks"],
         }
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = oracle_sample_rate(w, q, k, v, target_s=args.cpu_seconds)
+        if extra:
+            line["workloads"] = extra
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -480,19 +635,22 @@ def run_gate_only(args):
 
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args):
+    """The fp64 oracle as it stands, on the host cores, on the same workload: each step is one
+    sample of a fixed number of query tokens (the same sample size the CPU-baseline leg uses)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     w = wl.WORKLOADS[args.workload]
     q, k, v, cu = wl.make_inputs(w, seed=0, device="cpu")
+    sampler = OracleSampler(w, q, k, v, target_s=oracle_target_seconds(args))
     for _ in range(args.warmup):
-        oracle_sample_rate(w, q, k, v, target_s=min(2.0, args.cpu_seconds))
+        sampler.sample()
     vals = []
     t0 = time.perf_counter()
     last = None
     for _ in range(args.steps):
-        last = oracle_sample_rate(w, q, k, v, target_s=args.cpu_seconds / max(args.steps, 1))
+        last = sampler.sample()
         vals.append(last["value"])
     wall = time.perf_counter() - t0
     value = statistics.median(vals)
@@ -518,7 +676,9 @@ def main():
     ap.add_argument("--workload", default="llama8b_128k", choices=list(wl.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only --workload (skip the 1M and small-block sub-records)")
     ap.add_argument("--only", choices=["gate"], default=None,
                     help="time centroids + gate alone (1 GPU; for profiling)")
     args = ap.parse_args()

@@ -26,6 +26,8 @@ enum KernelClass {
 };
 
 std::atomic<long long> g_launches{0};
+// Limit of one pipeline wait inside the attention kernel (0 = the built-in 2 s).
+std::atomic<unsigned long long> g_wait_limit_ns{0};
 
 // ------------------------------------------------------------------------------- timing hooks
 // Timing starts enabled when the process sets MOBA_TIMING=1.
@@ -358,7 +360,7 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu
   for (const Chunk& c : P.chunks) {
     MOBA_LAUNCH(kRouteCount, s,
                 launch_route_count(idx, tb, P.T, Hq, Hkv, topk, P.NB, c.b0, c.nblk, c.T0, P.max_nb,
-                                   counts, s));
+                                   counts, status, s));
     MOBA_LAUNCH(kRouteScan, s, launch_route_scan(counts, NBK, cursor, tiles, n_tiles, s));
     MOBA_LAUNCH(kRouteScatter, s,
                 launch_route_scatter(idx, tb, P.T, Hq, Hkv, topk, P.NB, c.b0, c.nblk, c.T0,
@@ -375,6 +377,7 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu
     A.part_o = part_o; A.part_lse = part_lse; A.status = status;
     A.T = P.T; A.H = Hq; A.G = Hkv; A.d = d; A.B = block_size; A.topk = topk; A.NB = P.NB;
     A.b0 = c.b0; A.nblk = c.nblk; A.T0 = c.T0; A.scale = scale;
+    A.wait_ns = g_wait_limit_ns.load();
     const long long P256 = (block_size + kItemRows - 1) / kItemRows;
     const long long items = static_cast<long long>(P.max_tiles) + P256 * c.nblk * Hq;
     A.grid = static_cast<int>(std::min<long long>(sms, items));
@@ -384,6 +387,17 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu
                              c.ntok, o, lse, s));
   }
   return MOBA_OK;
+}
+
+int read_status_word(const void* word_dev, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int word = 0;
+  if (cudaMemcpyAsync(&word, word_dev, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOBA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOBA_ERR_CUDA;
+  if (word == 0) return MOBA_OK;
+  if (word == kDevTimeoutAttn || word == kDevDrainTimeout) return MOBA_ERR_TIMEOUT;
+  return MOBA_ERR_DEVICE_CHECK;
 }
 
 size_t workspace_bytes_for(int nseq, const int32_t* cu_host, int Hq, int Hkv, int d,
@@ -411,14 +425,12 @@ int moba_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu
 
 int moba_device_status(const void* workspace, void* stream) {
   if (!workspace) return MOBA_ERR_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int word = 0;
-  if (cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return MOBA_ERR_CUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return MOBA_ERR_CUDA;
-  if (word == 0) return MOBA_OK;
-  if (word == kDevTimeoutAttn) return MOBA_ERR_TIMEOUT;
-  return MOBA_ERR_DEVICE_CHECK;
+  return moba::read_status_word(workspace, stream);
+}
+
+unsigned long long moba_set_wait_limit_ns(unsigned long long ns) {
+  const unsigned long long was = g_wait_limit_ns.exchange(ns);
+  return was ? was : kWaitTimeoutNs;
 }
 
 int moba_timing_enable(int enable) {

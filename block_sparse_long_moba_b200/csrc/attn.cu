@@ -68,6 +68,7 @@ struct AttnArgs {
   int P2;                  // ceil(B / 256): diagonal items per (block, head)
   int n_diag;              // P2 * nblk * H diagonal items (some may be empty)
   float scale_log2;        // scale * log2(e)
+  unsigned long long wait_ns;  // limit of one pipeline wait (abort drains use kDrainTimeoutNs)
 };
 
 struct __align__(16) Item {
@@ -262,7 +263,7 @@ __global__ void __launch_bounds__(384, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // the swizzled layouts assume a 1024-byte aligned base: refuse to run otherwise
   if (smem_u32(smem64) & 1023u) {
-    if (tid == 0) atomicCAS(a.status, 0, kDevTimeoutAttn);
+    if (tid == 0) atomicCAS(a.status, 0, kDevSmemAlign);
     return;
   }
   if (tid == 0) {
@@ -308,7 +309,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = bars->tmem_base;
   const int n_routed = *a.n_routed;
   const int n_items = n_routed + a.n_diag;
-  const uint64_t TO = kWaitTimeoutNs;
+  const uint64_t TO = a.wait_ns;
   int* err = a.status;
   auto pop = [&](uint32_t lt, Item& it) -> bool {
     return ring_consume(ring, lt, it, abort_flag, err, TO);
@@ -347,13 +348,13 @@ __global__ void __launch_bounds__(384, 1)
         volatile int no_abort = 0;
         for (uint32_t x = 0; x < static_cast<uint32_t>(C::NK) && x < issued_k; ++x) {
           const uint32_t Jx = issued_k - 1 - x;
-          mbar_wait_bounded(&bars->k_full[Jx % C::NK], (Jx / C::NK) & 1, &no_abort, nullptr, 0,
-                            TO / 4);
+          mbar_wait_bounded(&bars->k_full[Jx % C::NK], (Jx / C::NK) & 1, &no_abort, err, kDevDrainTimeout,
+                            kDrainTimeoutNs);
         }
         for (uint32_t x = 0; x < static_cast<uint32_t>(C::NV) && x < issued_v; ++x) {
           const uint32_t Jx = issued_v - 1 - x;
-          mbar_wait_bounded(&bars->v_full[Jx % C::NV], (Jx / C::NV) & 1, &no_abort, nullptr, 0,
-                            TO / 4);
+          mbar_wait_bounded(&bars->v_full[Jx % C::NV], (Jx / C::NV) & 1, &no_abort, err, kDevDrainTimeout,
+                            kDrainTimeoutNs);
         }
       }
     } else if (warp == 1) {
@@ -444,7 +445,7 @@ __global__ void __launch_bounds__(384, 1)
         // after an abort, wait (bounded) until the MMAs already issued have finished with TMEM
         volatile int no_abort = 0;
         mma_commit_elect(&bars->drain);
-        mbar_wait_bounded(&bars->drain, 0, &no_abort, nullptr, 0, TO / 4);
+        mbar_wait_bounded(&bars->drain, 0, &no_abort, err, kDevDrainTimeout, kDrainTimeoutNs);
       }
     } else if (warp == 2) {
       // ------------------------------------------------------------------ Q rows
@@ -498,8 +499,8 @@ __global__ void __launch_bounds__(384, 1)
         volatile int no_abort = 0;
         for (uint32_t x = 0; x < static_cast<uint32_t>(C::QB) && x < issued; ++x) {
           const uint32_t l = issued - 1 - x;
-          mbar_wait_bounded(&bars->q_full[l % C::QB], (l / C::QB) & 1, &no_abort, nullptr, 0,
-                            TO / 4);
+          mbar_wait_bounded(&bars->q_full[l % C::QB], (l / C::QB) & 1, &no_abort, err, kDevDrainTimeout,
+                            kDrainTimeoutNs);
         }
       }
     } else {
@@ -781,7 +782,7 @@ __global__ void __launch_bounds__(384, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // the swizzled layouts assume a 1024-byte aligned base: refuse to run otherwise
   if (smem_u32(smem) & 1023u) {
-    if (tid == 0) atomicCAS(a.status, 0, kDevTimeoutAttn);
+    if (tid == 0) atomicCAS(a.status, 0, kDevSmemAlign);
     return;
   }
   if (tid == 0) {
@@ -816,7 +817,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = bars->tmem_base;
   const int n_routed = *a.n_routed;
   const int n_items = n_routed + a.n_diag;
-  const uint64_t TO = kWaitTimeoutNs;
+  const uint64_t TO = a.wait_ns;
   int* err = a.status;
 
   if (warp < 4) {
@@ -859,10 +860,13 @@ __global__ void __launch_bounds__(384, 1)
         for (uint32_t x = 0; x < 2; ++x) {
           if (JK > x) {
             const uint32_t Jx = JK - 1 - x;
-            mbar_wait_bounded(&bars->k_full[Jx & 1], (Jx >> 1) & 1, &no_abort, nullptr, 0, TO / 4);
+            mbar_wait_bounded(&bars->k_full[Jx & 1], (Jx >> 1) & 1, &no_abort, err,
+                              kDevDrainTimeout, kDrainTimeoutNs);
           }
         }
-        if (JV > 0) mbar_wait_bounded(&bars->v_full, (JV - 1) & 1, &no_abort, nullptr, 0, TO / 4);
+        if (JV > 0)
+          mbar_wait_bounded(&bars->v_full, (JV - 1) & 1, &no_abort, err, kDevDrainTimeout,
+                            kDrainTimeoutNs);
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------------ MMA issuer
@@ -935,7 +939,7 @@ __global__ void __launch_bounds__(384, 1)
       if (!ok) {
         volatile int no_abort = 0;
         mma_commit_elect(&bars->drain);
-        mbar_wait_bounded(&bars->drain, 0, &no_abort, nullptr, 0, TO / 4);
+        mbar_wait_bounded(&bars->drain, 0, &no_abort, err, kDevDrainTimeout, kDrainTimeoutNs);
       }
     } else {
       // ------------------------------------------------------------------ Q row gather
@@ -1000,7 +1004,8 @@ __global__ void __launch_bounds__(384, 1)
       if (!ok && half == 0 && lt > 0) {
         // after an abort, let the gathers still in flight land before the CTA exits (bounded)
         volatile int no_abort = 0;
-        mbar_wait_bounded(&bars->q_full, (lt - 1) & 1, &no_abort, nullptr, 0, TO / 4);
+        mbar_wait_bounded(&bars->q_full, (lt - 1) & 1, &no_abort, err, kDevDrainTimeout,
+                          kDrainTimeoutNs);
       }
     }
   } else {
@@ -1031,9 +1036,12 @@ __global__ void __launch_bounds__(384, 1)
       }
       float m_ref = -INFINITY, l_sum = 0.f;
       for (int j = 0; j < it.nsub; ++j, ++J) {
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[half], J & 1, abort_flag,
-                                                       err, kDevTimeoutAttn, TO));
-        if (!ok) break;
+        // A warp whose wait gives up does not leave on its own: the four warps of this half meet
+        // at named barriers, so the decision to leave is taken by all of them together at the
+        // next barrier (a warp that left alone would strand the other three there). Until then
+        // a warp that gave up computes on whatever S holds; its results are never used.
+        bool wok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[half], J & 1,
+                                                             abort_flag, err, kDevTimeoutAttn, TO));
         tc_fence_after();
         uint32_t sr[128];
         const int lim = limit - j * kTile;
@@ -1097,13 +1105,14 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 0; c < 64; c += 2) sr[c >> 1] = exp_pair(c);
         // P(J) reuses the shared P tile: PV(J-1) must be complete (it also fixes O^T for a rescale)
-        if (J > 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done, (J - 1) & 1, abort_flag,
-                                                         err, kDevTimeoutAttn, TO));
-          if (!ok) break;
-        }
+        if (J > 0 && wok)
+          wok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done, (J - 1) & 1,
+                                                          abort_flag, err, kDevTimeoutAttn, TO));
         s_alpha[q] = alpha;
-        if (named_bar_or(bar_id, 128, need && j > 0)) {
+        // one barrier answers both questions in the common case: nothing to rescale, no abort
+        if (named_bar_or(bar_id, 128, !wok || (need && j > 0))) {
+          ok = named_bar_and(bar_id, 128, wok);  // the same answer for every warp of the half
+          if (!ok) break;
           // some row of this half raised its max: scale this half's O^T columns (lane = d)
           tc_fence_after();
 #pragma unroll 1
@@ -1139,12 +1148,13 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (!ok) break;
       // ---- epilogue: O = O^T / l, transposed through the (now idle) P tile
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done, (J - 1) & 1, abort_flag, err,
-                                                     kDevTimeoutAttn, TO));
-      if (!ok) break;
+      const bool eok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done, (J - 1) & 1,
+                                                                 abort_flag, err, kDevTimeoutAttn,
+                                                                 TO));
       tc_fence_after();
       s_invl[q] = (valid && l_sum > 0.f) ? 1.f / l_sum : 0.f;
-      named_bar_sync(bar_id, 128);
+      ok = named_bar_and(bar_id, 128, eok);  // leave together or not at all
+      if (!ok) break;
       // thread `row` holds O^T lane d = row: columns are this half's 128 query rows
 #pragma unroll 1
       for (int c0 = 0; c0 < kTile; c0 += 32) {
@@ -1282,6 +1292,7 @@ cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream) {
   a.P2 = (L.B + kItemRows - 1) / kItemRows;
   a.n_diag = a.P2 * L.nblk * L.H;
   a.scale_log2 = L.scale * 1.4426950408889634f;
+  a.wait_ns = L.wait_ns > 0 ? L.wait_ns : kWaitTimeoutNs;
   const int grid = L.grid > 0 ? L.grid : 1;
   // setmaxnreg.inc would wait forever if the launch had fewer registers than the split assumes
   {

@@ -11,9 +11,16 @@ constexpr int kItemRows = 256;       // query rows per attention work item (two 
 constexpr int kMaxTopk = 64;
 constexpr int kMaxBlocksPerSeq = 32768;
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s per bounded device wait
+// After an abort, a CTA waits for its own copies and matrix products still in flight before it
+// exits. That drain has its own limit, independent of the pipeline-wait limit (which a caller
+// may shorten for diagnostics), so that a short pipeline limit never cuts a drain short.
+constexpr unsigned long long kDrainTimeoutNs = 2000000000ull;
 
 // Device status word codes (written with atomicCAS(word, 0, code); first failure wins).
-constexpr int kDevTimeoutAttn = 0x101;
+constexpr int kDevTimeoutAttn = 0x101;   // a pipeline wait ran out          -> MOBA_ERR_TIMEOUT
+constexpr int kDevDrainTimeout = 0x102;  // an abort drain ran out            -> MOBA_ERR_TIMEOUT
+constexpr int kDevBadRouting = 0x201;    // a routing row breaks its contract -> MOBA_ERR_DEVICE_CHECK
+constexpr int kDevSmemAlign = 0x301;     // dynamic shared memory misaligned  -> MOBA_ERR_DEVICE_CHECK
 
 // Block tables built on the device from cu_seqlens (workspace resident).
 struct BlockTables {

@@ -43,9 +43,11 @@ cudaError_t launch_gate_tc(const void* q, const float* cents, const int32_t* cu_
                            int max_nb, int T, int H, int G, int d, int B, int topk, int32_t* idx,
                            int* status, int num_sms, cudaStream_t stream);
 
+// Counts the routed entries per (kv head, block) and checks every routing row of the chunk
+// against its contract (kDevBadRouting in *status on the first bad row).
 cudaError_t launch_route_count(const int32_t* idx, const BlockTables& tb, int T, int H, int G,
                                int topk, int NB, int b0, int nblk, int T0, int max_nb,
-                               int* counts, cudaStream_t stream);
+                               int* counts, int* status, cudaStream_t stream);
 
 cudaError_t launch_route_scan(int* counts, int nbk, int* cursor, int4* tiles, int* n_tiles,
                               cudaStream_t stream);
@@ -76,6 +78,7 @@ struct AttnLaunch {
   int b0, nblk, T0;
   float scale;
   int grid;
+  unsigned long long wait_ns = 0;  // pipeline-wait limit; 0 = kWaitTimeoutNs
 };
 
 cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream);
@@ -91,6 +94,9 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu
                   int topk, float scale, const int32_t* block_idx_in, int32_t* block_idx_out,
                   void* o, float* lse, void* workspace, size_t workspace_bytes, void* stream,
                   size_t partial_budget);
+
+// Synchronises `stream`, reads the device status word at `word_dev` and maps it to a status.
+int read_status_word(const void* word_dev, void* stream);
 
 // Workspace bytes attn_fwd_impl needs with the given chunk budget (0 on invalid arguments).
 size_t workspace_bytes_for(int nseq, const int32_t* cu_host, int Hq, int Hkv, int d,

@@ -20,6 +20,8 @@
 //     array: serialise them.
 //   * The first call on each device looks up the array's device address (cudaGetSymbolAddress,
 //     with that device current). Make that first call before any stream capture begins.
+//   * The device status word of a call (a bounded wait that ran out, a routing row that broke
+//     its contract) sits at the start of the array; moba_noalloc_status reads it.
 #include <mutex>
 
 #include "../../include/moba.h"
@@ -70,4 +72,11 @@ extern "C" int moba_attn_fwd_noalloc(const void* q, const void* k, const void* v
   return moba::attn_fwd_impl(q, k, v, cu_seqlens_dev, cu_seqlens_host, nseq, Hq, Hkv, d,
                              block_size, topk, scale, nullptr, nullptr, o, lse, scratch,
                              MOBA_NOALLOC_SCRATCH_BYTES, stream, kNoallocPartialBudget);
+}
+
+extern "C" int moba_noalloc_status(void* stream) {
+  void* scratch = nullptr;
+  const int st = scratch_for_current_device(&scratch);
+  if (st != MOBA_OK) return st;
+  return moba::read_status_word(scratch, stream);
 }

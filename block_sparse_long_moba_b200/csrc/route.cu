@@ -80,31 +80,50 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
 }
 
 // Walk the routed (t, h, slot) triples of one (query block b, kv head g): slots j < i only.
+// The counting pass also checks each row against the routing contract the merge relies on: with
+// n = min(topk, i + 1), slots 0 .. n-2 hold strictly ascending past blocks (0 <= j < i), slot n-1
+// holds the current block i and the remaining slots hold -1. The diagonal tiles write slot n-1
+// and the merge reads slots 0 .. n-1, so a row that breaks this (e.g. a caller-supplied routing
+// with fewer blocks) would merge slots nobody wrote: it is reported as kDevBadRouting. Entries
+// outside 0 <= j < i are never counted or scattered, so a bad row cannot index out of bounds.
 template <bool kScatter>
 __global__ void __launch_bounds__(256) route_pass_kernel(
     const int32_t* __restrict__ idx, BlockTables tb, int T, int H, int G, int topk, int NB,
     int b0, int T0, int* __restrict__ counts, int* __restrict__ cursor,
-    int* __restrict__ entries) {
+    int* __restrict__ entries, int* __restrict__ status) {
   extern __shared__ int hist[];
   const int b = b0 + blockIdx.x, g = blockIdx.y;
   const int s = tb.blk_seq[b];
   const int base = tb.blk_off[s];
   const int i = b - base;
-  if (i == 0) return;
+  if (kScatter && i == 0) return;
   const int len = tb.blk_len[b], tstart = tb.blk_start[b];
   const int r = H / G;
   for (int x = threadIdx.x; x < i; x += blockDim.x) hist[x] = 0;
   __syncthreads();
   const int rows = r * len;
+  const int n = min(topk, i + 1);
+  bool bad = false;
   for (int row = threadIdx.x; row < rows; row += blockDim.x) {
     const int hh = row / len, t = tstart + row % len;
     const int32_t* rp = idx + (static_cast<size_t>(g * r + hh) * T + t) * topk;
+    int prev = -1;
     for (int slot = 0; slot < topk; ++slot) {
       const int j = __ldg(rp + slot);
+      if (!kScatter) {
+        bad |= slot < n - 1 ? (j <= prev || j >= i) : slot == n - 1 ? (j != i) : (j != -1);
+        prev = j;
+      }
       if (j >= 0 && j < i) atomicAdd(&hist[j], 1);
     }
   }
-  __syncthreads();
+  if (!kScatter) {
+    if (__syncthreads_or(bad) && threadIdx.x == 0 && status)
+      atomicCAS(status, 0, kDevBadRouting);
+    if (i == 0) return;
+  } else {
+    __syncthreads();
+  }
   int* gbucket = (kScatter ? cursor : counts) + static_cast<size_t>(g) * NB + base;
   for (int x = threadIdx.x; x < i; x += blockDim.x) {
     const int c = hist[x];
@@ -225,13 +244,13 @@ cudaError_t launch_plan(const int32_t* cu_dev, int nseq, int B, int NB, const Bl
 
 cudaError_t launch_route_count(const int32_t* idx, const BlockTables& tb, int T, int H, int G,
                                int topk, int NB, int b0, int nblk, int T0, int max_nb,
-                               int* counts, cudaStream_t stream) {
+                               int* counts, int* status, cudaStream_t stream) {
   const int smem = max_nb * 4;
   cudaError_t e = cudaFuncSetAttribute(route_pass_kernel<false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  route_pass_kernel<false><<<dim3(nblk, G), 256, smem, stream>>>(idx, tb, T, H, G, topk, NB, b0,
-                                                                 T0, counts, nullptr, nullptr);
+  route_pass_kernel<false><<<dim3(nblk, G), 256, smem, stream>>>(
+      idx, tb, T, H, G, topk, NB, b0, T0, counts, nullptr, nullptr, status);
   return cudaGetLastError();
 }
 
@@ -259,8 +278,8 @@ cudaError_t launch_route_scatter(const int32_t* idx, const BlockTables& tb, int 
   cudaError_t e = cudaFuncSetAttribute(route_pass_kernel<true>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  route_pass_kernel<true><<<dim3(nblk, G), 256, smem, stream>>>(idx, tb, T, H, G, topk, NB, b0,
-                                                                T0, nullptr, cursor, entries);
+  route_pass_kernel<true><<<dim3(nblk, G), 256, smem, stream>>>(
+      idx, tb, T, H, G, topk, NB, b0, T0, nullptr, cursor, entries, nullptr);
   return cudaGetLastError();
 }
 

@@ -24,7 +24,7 @@ KERNEL_CLASSES = ["centroid", "gate", "route_count", "route_scan", "route_scatte
 EXPORTS = ["moba_status_string", "moba_version", "moba_workspace_bytes", "moba_centroids",
            "moba_gate_topk", "moba_attn_fwd", "moba_device_status", "moba_timing_enable",
            "moba_timing_reset", "moba_timing_read", "moba_launch_count",
-           "moba_attn_fwd_noalloc"]
+           "moba_attn_fwd_noalloc", "moba_noalloc_status", "moba_set_wait_limit_ns"]
 
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -69,6 +69,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moba_launch_count.restype = L
     lib.moba_attn_fwd_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P, P, P]
     lib.moba_attn_fwd_noalloc.restype = I
+    lib.moba_noalloc_status.argtypes = [P]
+    lib.moba_noalloc_status.restype = I
+    lib.moba_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    lib.moba_set_wait_limit_ns.restype = ctypes.c_ulonglong
     _lib = lib
     return lib
 
@@ -86,6 +90,47 @@ def _stream(stream) -> ctypes.c_void_p:
 def _check(status: int, what: str):
     if status != 0:
         raise MobaError(status, what)
+
+
+_ANY_DEVICE = object()  # the device is checked separately (_current_device)
+
+
+def _bad(what: str, why: str):
+    raise MobaError(-1, f"{what}: {why}")
+
+
+def _want(what: str, name: str, t: Optional[torch.Tensor], dtype, shape=None, device=None):
+    """Checks one tensor argument before its pointer reaches the library: the kernels trust the
+    layout (dtype, contiguity, shape) and launch on the current device, so a mismatch here would
+    otherwise read or write the wrong memory."""
+    if t is None:
+        _bad(what, f"{name} is required")
+    if not torch.is_tensor(t):
+        _bad(what, f"{name} must be a torch tensor")
+    if t.dtype != dtype:
+        _bad(what, f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        _bad(what, f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        _bad(what, f"{name} must be contiguous")
+    if device is None:
+        if t.device.type != "cuda":
+            _bad(what, f"{name} must be a CUDA tensor, got {t.device}")
+    elif device is not _ANY_DEVICE and t.device != device:
+        _bad(what, f"{name} is on {t.device}, the call runs on {device}")
+
+
+def _current_device(what: str, t: torch.Tensor) -> torch.device:
+    if t.device.type != "cuda":
+        _bad(what, f"tensors must be CUDA tensors, got {t.device}")
+    cur = torch.device("cuda", torch.cuda.current_device())
+    if t.device != cur:
+        _bad(what, f"tensors are on {t.device} but the current device is {cur}")
+    return cur
+
+
+def _want_cu(what: str, cu_seqlens: torch.Tensor, nseq: int, device):
+    _want(what, "cu_seqlens", cu_seqlens, torch.int32, (nseq + 1,), device)
 
 
 def _host_cu(cu_seqlens_host) -> Tuple[ctypes.Array, int]:
@@ -109,11 +154,18 @@ def moba_workspace_bytes(cu_seqlens_host, hq: int, hkv: int, d: int, block_size:
 def moba_centroids(k: torch.Tensor, cu_seqlens: torch.Tensor, cu_seqlens_host, block_size: int,
                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Block centroids [NB, Hkv, d] fp32 of bf16 keys [T, Hkv, d]."""
+    what = "moba_centroids"
     arr, nseq = _host_cu(cu_seqlens_host)
+    if not torch.is_tensor(k) or k.dim() != 3:
+        _bad(what, "k must be a [T, Hkv, d] tensor")
     T, hkv, d = k.shape
+    _want(what, "k", k, torch.bfloat16, None, _ANY_DEVICE)
+    dev = _current_device(what, k)
+    _want_cu(what, cu_seqlens, nseq, dev)
     nb = num_blocks(list(arr), block_size)
     if out is None:
         out = torch.empty((nb, hkv, d), dtype=torch.float32, device=k.device)
+    _want(what, "out", out, torch.float32, (nb, hkv, d), dev)
     st = load_library().moba_centroids(_ptr(k), _ptr(cu_seqlens), arr, nseq, hkv, d, block_size,
                                        _ptr(out), _stream(stream))
     _check(st, "moba_centroids")
@@ -124,15 +176,40 @@ def moba_gate_topk(q: torch.Tensor, centroids: torch.Tensor, cu_seqlens: torch.T
                    cu_seqlens_host, block_size: int, topk: int,
                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Routing [Hq, T, topk] int32 (ascending local block ids, -1 padded)."""
+    what = "moba_gate_topk"
     arr, nseq = _host_cu(cu_seqlens_host)
+    if not torch.is_tensor(q) or q.dim() != 3 or not torch.is_tensor(centroids) or \
+            centroids.dim() != 3:
+        _bad(what, "q must be [T, Hq, d] and centroids [NB, Hkv, d]")
     T, hq, d = q.shape
     hkv = centroids.shape[1]
+    _want(what, "q", q, torch.bfloat16, None, _ANY_DEVICE)
+    dev = _current_device(what, q)
+    _want(what, "centroids", centroids, torch.float32,
+          (num_blocks(list(arr), block_size), hkv, d), dev)
+    _want_cu(what, cu_seqlens, nseq, dev)
     if out is None:
         out = torch.empty((hq, T, topk), dtype=torch.int32, device=q.device)
+    _want(what, "out", out, torch.int32, (hq, T, topk), dev)
     st = load_library().moba_gate_topk(_ptr(q), _ptr(centroids), _ptr(cu_seqlens), arr, nseq, hq,
                                        hkv, d, block_size, topk, _ptr(out), _stream(stream))
     _check(st, "moba_gate_topk")
     return out
+
+
+def _check_qkv(what, q, k, v, cu_seqlens, nseq):
+    """q [T, Hq, d], k and v [T, Hkv, d], all bf16, contiguous, on the current device."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not torch.is_tensor(t) or t.dim() != 3:
+            _bad(what, f"{name} must be a 3-D tensor")
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    _want(what, "q", q, torch.bfloat16, None, _ANY_DEVICE)
+    dev = _current_device(what, q)
+    _want(what, "k", k, torch.bfloat16, (T, hkv, d), dev)
+    _want(what, "v", v, torch.bfloat16, (T, hkv, d), dev)
+    _want_cu(what, cu_seqlens, nseq, dev)
+    return dev, T, hq, hkv, d
 
 
 def moba_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
@@ -142,16 +219,23 @@ def moba_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens:
                   o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                   workspace: Optional[torch.Tensor] = None, stream=None):
     """MoBA forward: returns (o [T,Hq,d] bf16, lse [Hq,T] fp32). Buffers may be passed in."""
+    what = "moba_attn_fwd"
     arr, nseq = _host_cu(cu_seqlens_host)
-    T, hq, d = q.shape
-    hkv = k.shape[1]
+    dev, T, hq, hkv, d = _check_qkv(what, q, k, v, cu_seqlens, nseq)
     if scale is None:
         scale = d ** -0.5
+    for name, t in (("block_idx_in", block_idx_in), ("block_idx_out", block_idx_out)):
+        if t is not None:
+            _want(what, name, t, torch.int32, (hq, T, topk), dev)
     lib = load_library()
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((hq, T), dtype=torch.float32, device=q.device)
+    _want(what, "o", o, torch.bfloat16, (T, hq, d), dev)
+    _want(what, "lse", lse, torch.float32, (hq, T), dev)
+    if workspace is not None:
+        _want(what, "workspace", workspace, torch.uint8, None, dev)
     if workspace is None:
         nbytes = int(lib.moba_workspace_bytes(nseq, arr, hq, hkv, d, block_size, topk))
         if nbytes == 0 and T > 0:
@@ -172,15 +256,17 @@ def moba_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     """moba_attn_fwd without a workspace: the library's static scratch array is used instead
     (for callers that cannot allocate device memory; see include/moba.h). The outputs may be
     passed in so that the call itself allocates nothing."""
+    what = "moba_attn_fwd_noalloc"
     arr, nseq = _host_cu(cu_seqlens_host)
-    T, hq, d = q.shape
-    hkv = k.shape[1]
+    dev, T, hq, hkv, d = _check_qkv(what, q, k, v, cu_seqlens, nseq)
     if scale is None:
         scale = d ** -0.5
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((hq, T), dtype=torch.float32, device=q.device)
+    _want(what, "o", o, torch.bfloat16, (T, hq, d), dev)
+    _want(what, "lse", lse, torch.float32, (hq, T), dev)
     st = load_library().moba_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), arr,
                                               nseq, hq, hkv, d, block_size, topk,
                                               ctypes.c_float(scale), _ptr(o), _ptr(lse),
@@ -191,6 +277,17 @@ def moba_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 
 def moba_device_status(workspace: torch.Tensor, stream=None) -> int:
     return int(load_library().moba_device_status(_ptr(workspace), _stream(stream)))
+
+
+def moba_noalloc_status(stream=None) -> int:
+    """Status word of the last moba_attn_fwd_noalloc call on the current device (synchronises)."""
+    return int(load_library().moba_noalloc_status(_stream(stream)))
+
+
+def set_wait_limit_ns(ns: int) -> int:
+    """Diagnostics: limit of one pipeline wait in the attention kernel (0 = built-in 2 s);
+    returns the previous limit."""
+    return int(load_library().moba_set_wait_limit_ns(ctypes.c_ulonglong(int(ns))))
 
 
 def timing_enable(on: bool = True):

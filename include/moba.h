@@ -55,7 +55,8 @@ typedef enum {
   MOBA_ERR_UNSUPPORTED = -2,  /* valid but outside the supported shapes or device             */
   MOBA_ERR_WORKSPACE = -3,    /* workspace smaller than moba_workspace_bytes()                */
   MOBA_ERR_CUDA = -4,         /* a CUDA runtime / driver call or a kernel launch failed       */
-  MOBA_ERR_DEVICE_CHECK = -5, /* a device-side check failed (see moba_device_status)          */
+  MOBA_ERR_DEVICE_CHECK = -5, /* a device-side check failed, e.g. a routing row that breaks its
+                                 contract (see moba_device_status)                            */
   MOBA_ERR_TIMEOUT = -6       /* a bounded device-side wait ran out (see moba_device_status)  */
 } moba_status;
 
@@ -105,8 +106,14 @@ int moba_gate_topk(const void* q, const float* centroids, const int32_t* cu_seql
  *   o[t, h, :] = sum_u softmax_u(scale * q[t,h] . k[u,g]) v[u, g] over the keys u of the selected
  *   blocks (keys <= t inside the current block); lse[h, t] = log sum_u exp(scale * q . k_u).
  * block_idx_in : nullable. When given (device int32 [Hq, T, topk], same format as the gate's
- *                output), this routing is used and no centroid / gate work runs. The caller
- *                guarantees it is valid (current block present, no future block, ascending).
+ *                output), this routing is used and no centroid / gate work runs. Every row must
+ *                hold exactly n = min(topk, i + 1) blocks for a query in local block i: slots
+ *                0 .. n-2 strictly ascending past blocks (0 <= j < i), slot n-1 the current block
+ *                i, the other slots -1. The partial results of a row live in the slots of its
+ *                blocks and the merge reads slots 0 .. n-1, so a row with fewer blocks would mix
+ *                in slots nobody wrote. Rows are checked on the device: a row that breaks the
+ *                contract makes moba_device_status return MOBA_ERR_DEVICE_CHECK (the outputs of
+ *                that call are then undefined; out-of-range entries are never dereferenced).
  * block_idx_out: nullable. When given, receives the routing that was used.
  * workspace    : device buffer of at least moba_workspace_bytes(...) bytes, 256-byte aligned.
  */
@@ -134,8 +141,7 @@ int moba_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu
  *     must be serialised by the caller.
  *   - The first call on a device looks up the array's device address (with that device
  *     current); make that first call before any stream capture begins.
- *   - Device-side status (bounded waits) is not readable through moba_device_status for this
- *     entry point; a failed wait leaves the outputs undefined.
+ *   - The status word of the last call lives in the array; read it with moba_noalloc_status.
  */
 #define MOBA_NOALLOC_SCRATCH_BYTES (64u << 20)
 int moba_attn_fwd_noalloc(const void* q, const void* k, const void* v,
@@ -144,11 +150,30 @@ int moba_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                           float* lse, void* stream);
 
 /*
+ * Synchronises `stream`, then reads the status word of the last moba_attn_fwd_noalloc call on
+ * the current device (the word sits in the library's static scratch array): MOBA_OK,
+ * MOBA_ERR_TIMEOUT or MOBA_ERR_DEVICE_CHECK, as for moba_device_status. Calls that overlap on
+ * the GPU share the word like the rest of the array.
+ */
+int moba_noalloc_status(void* stream);
+
+/*
  * Synchronises `stream`, then reads the status word a moba_attn_fwd call left in `workspace`:
- * MOBA_OK, or MOBA_ERR_TIMEOUT when a bounded device wait ran out (the outputs of that call are
- * then undefined). The word is cleared by the next moba_attn_fwd on the same workspace.
+ * MOBA_OK; MOBA_ERR_TIMEOUT when a bounded device wait (or the drain after it) ran out; or
+ * MOBA_ERR_DEVICE_CHECK when a routing row broke its contract or the kernel found its shared
+ * memory misaligned. Outputs of a call with a status other than MOBA_OK are undefined. The word
+ * is cleared by the next moba_attn_fwd on the same workspace; the first failure of a call wins.
  */
 int moba_device_status(const void* workspace, void* stream);
+
+/*
+ * Diagnostics: sets the limit of one pipeline wait inside the attention kernel for later calls
+ * (process-wide; ns = 0 restores the built-in 2 s) and returns the previous limit. A short limit
+ * makes a wait run out on purpose, so that a test can see the abort path report
+ * MOBA_ERR_TIMEOUT while the context stays usable; after an abort each CTA still waits for its
+ * own copies and matrix products in flight, under a separate fixed 2 s limit, before it exits.
+ */
+unsigned long long moba_set_wait_limit_ns(unsigned long long ns);
 
 /*
  * Instrumentation (off by default; on from the start when the environment sets MOBA_TIMING=1).

@@ -17,7 +17,7 @@ gradients of step 4 with the routing held fixed: attention_backward):
   4. Attention is exact softmax attention over the keys of the selected blocks, restricted to
      key positions <= the query inside the current block [same page, "Approach": causal].
 
-Readings where the pages are silent (each one listed in the design doc):
+Readings where the pages are silent (the plainest reading of each, stated here):
   * centroid = mean over the keys actually present (a ragged last block averages fewer keys);
   * gate score = unscaled q . c in fp64; ties go to the lower block index;
   * the current block counts toward k; with k-1 >= i every block 0..i is selected;
@@ -114,6 +114,9 @@ class Routing:
     idx: np.ndarray      # [H, n, topk] int32, ascending local block ids, -1 padded
     margin: np.ndarray   # [H, n] relative gap between last selected and first unselected past score
     boundary: np.ndarray  # [H, n] the first unselected past score (nan if every past block is kept)
+    # [H, n] max over those two blocks of sum_i |q_i c_i|: the size of the terms each score sums,
+    # which bounds the rounding error of a score evaluated in floating point (0 if none)
+    magnitude: np.ndarray
 
 
 def select_blocks(q, cents: np.ndarray, cu_seqlens, block_size, topk, tokens=None) -> Routing:
@@ -138,6 +141,7 @@ def select_blocks(q, cents: np.ndarray, cu_seqlens, block_size, topk, tokens=Non
     idx = np.full((H, n, k), -1, np.int32)
     margin = np.full((H, n), np.inf)
     boundary = np.full((H, n), np.nan)
+    magnitude = np.zeros((H, n))
     # group query tokens by (sequence, local block): they share the same candidate blocks
     keys = s_of * (1 << 32) + i_of
     for key in np.unique(keys):
@@ -162,13 +166,18 @@ def select_blocks(q, cents: np.ndarray, cu_seqlens, block_size, topk, tokens=Non
             a = sc[m, order[:, k - 2]] if k >= 2 else np.full(len(rows), np.inf)
             bnd = sc[m, order[:, k - 1]]
             boundary[h, rows] = bnd
+            absq = np.abs(qf[:, h, :])                                  # [m, d]
+            mag_b = np.einsum("md,md->m", absq, np.abs(c_past[order[:, k - 1]]))
+            mag_a = (np.einsum("md,md->m", absq, np.abs(c_past[order[:, k - 2]])) if k >= 2
+                     else np.zeros(len(rows)))
+            magnitude[h, rows] = np.maximum(mag_a, mag_b)
             if k >= 2:
                 denom = np.maximum(np.abs(a), np.abs(bnd))
                 with np.errstate(invalid="ignore", divide="ignore"):
                     margin[h, rows] = np.where(denom > 0, (a - bnd) / denom, 0.0)
             else:
                 margin[h, rows] = np.inf
-    return Routing(tokens, idx, margin, boundary)
+    return Routing(tokens, idx, margin, boundary, magnitude)
 
 
 def gate_scores(q, cents: np.ndarray, cu_seqlens, block_size, token: int, head: int) -> np.ndarray:
@@ -242,10 +251,10 @@ def attention_backward(q, k, v, cu_seqlens, block_size, idx_full, scale, d_out) 
 
     MoBA is trained end to end through its block-sparse attention [MoBA README, "Introducing
     MoBA": trainable block sparse attention]; the top-k gate itself is piecewise constant in q and
-    the centroids, so no gradient flows through the selection (the reading of SURVEY row f1,
-    listed in the design doc). For every row (t, h) over its attended keys u (the keys of its selected
-    blocks, causal inside its own block), with z_u = scale q.k_u, p_u = exp(z_u - LSE) and
-    o = sum_u p_u v_u:
+    the centroids, so no gradient flows through the selection, as in top-k mixture-of-experts
+    routing (the pages are silent on this; it is the plainest reading). For every row (t, h)
+    over its attended keys u (the keys of its selected blocks, causal inside its own block), with
+    z_u = scale q.k_u, p_u = exp(z_u - LSE) and o = sum_u p_u v_u:
       dV[u] += p_u dO;  dP_u = dO . v_u;  D = dO . o;  dS_u = p_u (dP_u - D);
       dQ += scale sum_u dS_u k_u;  dK[u] += scale dS_u q.
     Keys and values of kv head g collect the terms of all query heads of its group. idx_full:

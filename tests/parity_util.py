@@ -8,12 +8,21 @@ from oracle import moba_ref as ref
 
 # Tolerances of the forward pass: |O - O_ref| <= O_ATOL + O_RTOL |O_ref| (elementwise, O read
 # back from bf16 as fp32), |LSE - LSE_ref| <= LSE_ATOL. Gate near-tie band: rows whose last
-# selected and first unselected past scores differ by less than TIE_REL (relative) may pick
-# either block; attention is then checked on the GPU's own selection.
+# selected and first unselected past scores a, b differ by less than
+#   max(TIE_REL * max(|a|, |b|), TIE_COND * M),   M = max over the two blocks of sum_i |q_i c_i|,
+# may pick either block; attention is then checked on the GPU's own selection. The first term is
+# the stated relative band. The second is the rounding of a score computed in fp32 arithmetic:
+# the kernel's split-bf16 centroids leave a residual below 2^-17 of each term and fp32
+# accumulation over d <= 128 terms adds below 128 * 2^-24 = 2^-17, so one score is within 2^-16 M
+# and a difference of two within 2^-15 M; TIE_COND doubles that. The second term only matters
+# when the two scores nearly cancel (|a|, |b| much smaller than M). TIE_ROWS_MAX bounds the share
+# of checked rows that may be excused as near ties on the full-size workloads.
 O_ATOL = 1e-2
 O_RTOL = 1e-2
 LSE_ATOL = 1e-3
 TIE_REL = 1e-4
+TIE_COND = 2.0 ** -14
+TIE_ROWS_MAX = 1e-3
 
 
 def check_routing(q_cpu, cents64, cu, B, topk, tokens, idx_gpu_rows, *, allow_ties=True):
@@ -38,13 +47,13 @@ def check_routing(q_cpu, cents64, cu, B, topk, tokens, idx_gpu_rows, *, allow_ti
         assert sel == sorted(set(sel)), (h, t, got)
         assert i in sel and max(sel) == i, (h, t, got)
         assert len(sel) == min(topk, i + 1), (h, t, got)
-        assert allow_ties and rt.margin[h, nn] < TIE_REL, (
-            f"routing mismatch outside the tie band: head {h} token {t} gpu {got} "
-            f"oracle {list(rt.idx[h, nn])} margin {rt.margin[h, nn]}")
         scores = ref.gate_scores(q_cpu, cents64, cu, B, t, int(h))
         order = np.sort(scores)[::-1]
         a, b = order[topk - 2], order[topk - 1]
-        tol = TIE_REL * max(abs(a), abs(b))
+        tol = max(TIE_REL * max(abs(a), abs(b)), TIE_COND * rt.magnitude[h, nn])
+        assert allow_ties and a - b <= tol, (
+            f"routing mismatch outside the tie band: head {h} token {t} gpu {got} "
+            f"oracle {list(rt.idx[h, nn])} margin {rt.margin[h, nn]} gap {a - b} band {tol}")
         past = [x for x in sel if x != i]
         unchosen = [j for j in range(i) if j not in past]
         assert all(scores[j] >= a - tol for j in past), (h, t, got)

@@ -37,6 +37,49 @@ def test_workload_flops_of_the_headline_configs():
     assert abs(bench.useful_flops(wl.WORKLOADS["llama8b_1m"]) / 1e12 - 791.1) < 0.1
 
 
+@pytest.mark.parametrize("cu,hq,hkv,d,B,topk", [
+    ([0, 1000], 2, 1, 64, 128, 3),
+    ([0, 300, 300, 1111], 4, 2, 128, 64, 5),
+    ([0, 2500], 2, 2, 64, 256, 4),
+    ([0, 9000], 2, 1, 128, 4096, 2),
+])
+def test_executed_flops_count_the_kernel_items(cu, hq, hkv, d, B, topk):
+    """Executed tile FLOPs by brute force: build every (kv head, past block) list from the
+    oracle's routing, cut it into 256-row items, add the diagonal items, and count 128 x 128
+    sub-tile pairs the way the kernels issue them (both halves at d = 128; at d = 64 one half for
+    items of at most 128 rows)."""
+    w = wl.custom(cu, hq, hkv, d, B, topk)
+    q, k, v, _ = wl.make_inputs(w, device="cpu")
+    rt = ref.select_blocks(q, ref.centroids(k, cu, B), cu, B, topk)
+    bt = ref.block_table(cu, B)
+    s_of, i_of = ref.token_position(cu, B, np.arange(cu[-1]))
+    r = hq // hkv
+    lists = {}
+    for h in range(hq):
+        for t in range(cu[-1]):
+            for j in rt.idx[h, t]:
+                if 0 <= j < i_of[t]:
+                    key = (h // r, int(bt.blk_off[s_of[t]]) + int(j))
+                    lists[key] = lists.get(key, 0) + 1
+
+    def rows_run(n):
+        return 256 if (d == 128 or n > 128) else 128
+
+    tiles = 0
+    for (g, b), c in lists.items():
+        nsub = -(-(int(bt.end[b]) - int(bt.start[b])) // 128)
+        for x in range(0, c, 256):
+            tiles += rows_run(min(256, c - x)) * nsub
+    for b in range(bt.num_blocks):
+        n = int(bt.end[b]) - int(bt.start[b])
+        for q0 in range(0, n, 256):
+            rows = min(256, n - q0)
+            tiles += hq * rows_run(rows) * -(-(q0 + rows) // 128)
+    got = bench.executed_flops(w, torch.as_tensor(rt.idx))
+    assert got == 4.0 * d * 128 * tiles
+    assert got >= bench.useful_flops(w)
+
+
 def test_job_throughput_is_weak_scaling():
     assert bench.job_throughput(1, 131072, 100.0) == pytest.approx(1.31072e6)
     assert bench.job_throughput(4, 131072, 100.0) == pytest.approx(4 * 1.31072e6)

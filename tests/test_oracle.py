@@ -2,8 +2,9 @@
 
 Each test ties one part of the oracle to something other than itself:
   * centroid      -> closed form on constructed keys (mean, ragged tail);
-  * gate          -> a constructed case with a hand-derived answer, ties, and brute-force subset
-                     enumeration on random inputs;
+  * gate          -> a constructed case with a hand-derived answer, ties, brute-force subset
+                     enumeration on random inputs, and hand-derived near-tie fields (margin,
+                     boundary) and per-head scores of a GQA layout;
   * full limit    -> with topk >= #blocks MoBA is causal attention: textbook formula and torch SDPA
                      in float64 (MoBA README, "Seamlessly Transition between Full and Sparse");
   * topk = 1      -> block-diagonal causal (local) attention;
@@ -105,6 +106,96 @@ def test_gate_ties_go_to_lower_block():
     t = 5 * B
     assert list(rt.idx[0, t]) == [0, 1, 5]      # four blocks score 2: the two lowest win
     assert rt.margin[0, t] == 0.0                # exact tie at the boundary
+
+
+def test_gate_margin_and_boundary_hand_derived():
+    """The near-tie fields of a row with distinct scores, worked out by hand.
+
+    Past scores of block 7 (head 0, q = e_1): w[0..6] = 3, -1, 5, 0, 2, 7, 1. With topk = 4 the
+    three best past blocks score 7, 5, 3; the first unselected scores 2, so
+    margin = (3 - 2) / max(|3|, |2|) = 1/3 and boundary = 2. Head 1 (q = -e_1) sees -w: the three
+    best are 1, 0, -1, the first unselected -2: margin = (-1 - (-2)) / 2 = 1/2, boundary = -2.
+    """
+    B = 4
+    w = [3, -1, 5, 0, 2, 7, 1, 4]
+    k = _const_block_keys(w, B)
+    T = k.shape[0]
+    c = ref.centroids(k, [0, T], B)
+    q = np.zeros((T, 2, 4), np.float32)
+    q[:, 0, 0] = 1.0
+    q[:, 1, 0] = -1.0
+    rt = ref.select_blocks(q, c, [0, T], B, 4)
+    t = 7 * B + 2
+    assert rt.margin[0, t] == pytest.approx(1.0 / 3.0, abs=1e-15)
+    assert rt.boundary[0, t] == 2.0
+    assert rt.margin[1, t] == pytest.approx(0.5, abs=1e-15)
+    assert rt.boundary[1, t] == -2.0
+    # magnitude: q = +-e_1, so sum_i |q_i c_i| of a block is |w_j|: max(|3|, |2|) and max(1, 2)
+    assert rt.magnitude[0, t] == 3.0 and rt.magnitude[1, t] == 2.0
+    # block 5 (past 3, -1, 5, 0, 2; top-3 = 5, 3, 2; next 0): margin (2 - 0) / 2 = 1
+    t5 = 5 * B
+    assert rt.margin[0, t5] == pytest.approx(1.0, abs=1e-15)
+    assert rt.boundary[0, t5] == 0.0
+    # every past block kept (k - 1 >= i): no boundary, no tie possible
+    assert np.isnan(rt.boundary[0, 3 * B]) and rt.margin[0, 3 * B] == np.inf
+    # a positive rescale of q scales the boundary and the magnitude, not the (relative) margin
+    rt2 = ref.select_blocks(2.0 * q, c, [0, T], B, 4)
+    assert rt2.boundary[0, t] == 4.0 and rt2.magnitude[0, t] == 6.0
+    assert rt2.margin[0, t] == pytest.approx(1.0 / 3.0, abs=1e-15)
+    # topk = 1 selects no past block: margin is infinite whatever the scores
+    rt1 = ref.select_blocks(q, c, [0, T], B, 1)
+    assert rt1.margin[0, t] == np.inf
+
+
+def test_gate_magnitude_sums_absolute_terms():
+    """magnitude sums |q_i| |c_i| over the dimensions: scores that cancel keep a large magnitude.
+    Block j's keys are (a_j, -a_j) in two dimensions and q = (1, 1), so every score is 0 while the
+    magnitude of block j is 2 |a_j|."""
+    B = 2
+    a = [1.0, 3.0, 2.0, 0.5, 4.0]
+    T = len(a) * B
+    k = np.zeros((T, 1, 2), np.float32)
+    for j, aj in enumerate(a):
+        k[j * B:(j + 1) * B, 0, 0] = aj
+        k[j * B:(j + 1) * B, 0, 1] = -aj
+    q = np.ones((T, 1, 2), np.float32)
+    c = ref.centroids(k, [0, T], B)
+    rt = ref.select_blocks(q, c, [0, T], B, 3)
+    t = 4 * B
+    # all four past scores are 0: ties go to the lower blocks, so 0 and 1 are kept, 2 is next
+    assert list(rt.idx[0, t]) == [0, 1, 4]
+    assert rt.boundary[0, t] == 0.0 and rt.margin[0, t] == 0.0
+    assert rt.magnitude[0, t] == max(2 * a[1], 2 * a[2])
+
+
+def test_gate_scores_hand_derived_gqa():
+    """gate_scores of a GQA layout (Hq = 4, Hkv = 2): query head h reads kv head h // 2.
+
+    Keys are constant inside each block: kv head 0 carries w0[j] e_1, kv head 1 carries w1[j] e_1,
+    and query head h is (h + 1) e_1, so the score of past block j is (h + 1) * w_{h // 2}[j].
+    """
+    B, d = 4, 4
+    w0 = [1.0, -2.0, 3.0, 0.5, 4.0]
+    w1 = [-1.0, 6.0, 0.25, 2.0, -3.0]
+    T = len(w0) * B
+    k = np.zeros((T, 2, d), np.float32)
+    for j in range(len(w0)):
+        k[j * B:(j + 1) * B, 0, 0] = w0[j]
+        k[j * B:(j + 1) * B, 1, 0] = w1[j]
+    q = np.zeros((T, 4, d), np.float32)
+    for h in range(4):
+        q[:, h, 0] = h + 1
+    c = ref.centroids(k, [0, T], B)
+    t = 4 * B + 1  # block 4: past blocks 0..3
+    for h in range(4):
+        want = [(h + 1) * wj for wj in (w0 if h < 2 else w1)[:4]]
+        np.testing.assert_array_equal(ref.gate_scores(q, c, [0, T], B, t, h), want)
+    # varlen: the second sequence's block 1 scores only that sequence's block 0
+    cu = [0, 2 * B, 4 * B]
+    c2 = ref.centroids(k[:4 * B], cu, B)
+    s = ref.gate_scores(q[:4 * B], c2, cu, B, 3 * B, 3)
+    np.testing.assert_array_equal(s, [4 * w1[2]])
+    assert ref.gate_scores(q, c, [0, T], B, 2, 0).shape == (0,)  # block 0 has no past
 
 
 def test_gate_brute_force_random():

@@ -8,6 +8,7 @@ from tests import test_oracle as pins
 _orig_centroids = ref.centroids
 _orig_select = ref.select_blocks
 _orig_attention = ref.attention
+_orig_gate_scores = ref.gate_scores
 
 
 def _sum_not_mean(k, cu, B):
@@ -45,11 +46,54 @@ def _negated_gate(q, cents, cu, B, topk, tokens=None):
     return _orig_select(q, -cents, cu, B, topk, tokens)
 
 
+def _margin_off_by_one(q, cents, cu, B, topk, tokens=None):
+    # near-tie fields taken one position too deep in the score order: the k-th and (k+1)-th best
+    # past scores instead of the (k-1)-th and k-th
+    rt = _orig_select(q, cents, cu, B, topk, tokens)
+    H, G = q.shape[1], cents.shape[1]
+    bt = ref.block_table(cu, B)
+    s_of, i_of = ref.token_position(cu, B, rt.tokens)
+    for n, t in enumerate(rt.tokens):
+        s, i = int(s_of[n]), int(i_of[n])
+        if topk - 1 >= i or topk < 2:
+            continue
+        for h in range(H):
+            qf = ref.to_f64(q[int(t):int(t) + 1])[0, h]
+            sc = cents[int(bt.blk_off[s]):int(bt.blk_off[s]) + i, h // (H // G)] @ qf
+            order = np.argsort(-sc, kind="stable")
+            a = sc[order[topk - 1]]
+            b = sc[order[topk]] if topk < i else np.nan
+            rt.boundary[h, n] = b
+            den = max(abs(a), abs(b)) if not np.isnan(b) else 1.0
+            rt.margin[h, n] = (a - b) / den if den > 0 else 0.0
+    return rt
+
+
+def _gate_scores_gqa_modulo(q, cents, cu, B, token, head):
+    # wrong head grouping in the per-row scores: kv head h % G instead of h // (H/G)
+    G = cents.shape[1]
+    H = q.shape[1]
+    perm_head = (head % G) * (H // G)  # a head of the group the modulo map picks
+    return _orig_gate_scores(q, cents, cu, B, token, perm_head) * (head + 1) / (perm_head + 1)
+
+
+def _magnitude_of_the_sum(q, cents, cu, B, topk, tokens=None):
+    # magnitude taken as |sum_i q_i c_i| (the score itself) instead of sum_i |q_i c_i|
+    rt = _orig_select(q, cents, cu, B, topk, tokens)
+    rt.magnitude = np.where(np.isnan(rt.boundary), 0.0,
+                            np.maximum(np.abs(rt.boundary),
+                                       np.abs(rt.boundary) * (1 + np.nan_to_num(rt.margin))))
+    return rt
+
+
 @pytest.mark.parametrize("target,fake,pin", [
     ("centroids", _sum_not_mean, pins.test_centroid_closed_form_with_ragged_tail),
     ("select_blocks", _negated_gate, pins.test_gate_constructed_case),
     ("select_blocks", _gqa_modulo, pins.test_gate_brute_force_random),
     ("attention", _no_causal_cut, pins.test_topk1_is_block_diagonal_causal),
+    ("select_blocks", _margin_off_by_one, pins.test_gate_margin_and_boundary_hand_derived),
+    ("gate_scores", _gate_scores_gqa_modulo, pins.test_gate_scores_hand_derived_gqa),
+    ("select_blocks", _magnitude_of_the_sum, pins.test_gate_magnitude_sums_absolute_terms),
 ])
 def test_pin_catches_planted_mistake(monkeypatch, target, fake, pin):
     monkeypatch.setattr(ref, target, fake)
