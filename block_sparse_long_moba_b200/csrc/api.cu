@@ -20,9 +20,10 @@ using namespace moba;
 namespace {
 
 constexpr size_t kPartialBudgetBytes = 16ull << 30;  // per-chunk partial outputs + routing lists
-constexpr int kNumClasses = 9;
+constexpr int kNumClasses = 10;
 enum KernelClass {
-  kCentroid = 0, kGate, kRouteCount, kRouteScan, kRouteScatter, kAttn, kMerge, kPlan, kDensify
+  kCentroid = 0, kGate, kRouteCount, kRouteScan, kRouteScatter, kAttn, kMerge, kPlan, kDensify,
+  kDecode
 };
 
 std::atomic<long long> g_launches{0};
@@ -56,7 +57,7 @@ Timing& timing() { static Timing t; return t; }
 const char* const kClassNames[kNumClasses] = {"moba_centroids", "moba_gate", "moba_route_count",
                                                "moba_route_scan", "moba_route_scatter",
                                                "moba_attention", "moba_merge", "moba_plan",
-                                               "moba_densify"};
+                                               "moba_densify", "moba_decode"};
 
 // Brackets one kernel launch: an NVTX range named for its class (seen by profilers; a no-op
 // otherwise) and, when timing is enabled, CUDA events on the launching stream.
@@ -253,6 +254,30 @@ size_t moba_workspace_bytes(int nseq, const int32_t* cu_seqlens_host, int Hq, in
   return layout_of(P, nseq, Hq, Hkv, d, topk).total;
 }
 
+int moba_centroids_kconv(const void* k, const float* conv_w, int conv_width,
+                         const int32_t* cu_dev, const int32_t* cu_host, int nseq, int Hkv, int d,
+                         int block_size, float* centroids, void* stream) {
+  if (!conv_w || !aligned16(conv_w)) return MOBA_ERR_ARG;
+  if (conv_width < 1) return MOBA_ERR_ARG;
+  if (conv_width > kMaxKconvWidth) return MOBA_ERR_UNSUPPORTED;
+  int st = check_cu(nseq, cu_host);
+  if (st != MOBA_OK) return st;
+  if (Hkv < 1 || block_size < 1) return MOBA_ERR_ARG;
+  if (d != 64 && d != 128) return MOBA_ERR_UNSUPPORTED;
+  if (block_size % 64 != 0) return MOBA_ERR_UNSUPPORTED;
+  Plan P;
+  if ((st = make_plan(nseq, cu_host, Hkv, Hkv, d, block_size, 1, &P)) != MOBA_OK) return st;
+  if (P.T == 0 || P.NB == 0) return MOBA_OK;
+  if (!k || !cu_dev || !centroids || !aligned16(k) || !aligned16(centroids)) return MOBA_ERR_ARG;
+  int sms = 0;
+  if ((st = device_check(&sms)) != MOBA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MOBA_LAUNCH(kCentroid, s,
+              launch_centroids(k, cu_dev, nseq, P.max_nb, Hkv, d, block_size, P.NB, sms, centroids,
+                               s, conv_w, conv_width));
+  return MOBA_OK;
+}
+
 int moba_centroids(const void* k, const int32_t* cu_dev, const int32_t* cu_host, int nseq,
                    int Hkv, int d, int block_size, float* centroids, void* stream) {
   int st = check_cu(nseq, cu_host);
@@ -302,9 +327,11 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu
                   const int32_t* cu_host, int nseq, int Hq, int Hkv, int d, int block_size,
                   int topk, float scale, const int32_t* block_idx_in, int32_t* block_idx_out,
                   void* o, float* lse, void* workspace, size_t workspace_bytes, void* stream,
-                  size_t partial_budget) {
+                  size_t partial_budget, const float* conv_w, int conv_width) {
   int st = check_cu(nseq, cu_host);
   if (st != MOBA_OK) return st;
+  if (conv_w && (!aligned16(conv_w) || conv_width < 1)) return MOBA_ERR_ARG;
+  if (conv_w && conv_width > kMaxKconvWidth) return MOBA_ERR_UNSUPPORTED;
   if ((st = check_shape(Hq, Hkv, d, block_size, topk)) != MOBA_OK) return st;
   if (!(scale > 0.f) || scale > 1e30f) return MOBA_ERR_ARG;
   Plan P;
@@ -346,7 +373,8 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu
   if (!idx) {
     int32_t* idx_w = block_idx_out ? block_idx_out : at<int32_t>(workspace, L.idx);
     MOBA_LAUNCH(kCentroid, s,
-                launch_centroids(k, cu_dev, nseq, P.max_nb, Hkv, d, block_size, P.NB, sms, cents, s));
+                launch_centroids(k, cu_dev, nseq, P.max_nb, Hkv, d, block_size, P.NB, sms, cents, s,
+                                 conv_w, conv_width));
     MOBA_LAUNCH(kGate, s,
                 run_gate(q, cents, cu_dev, cu_host, nseq, P.max_nb, P.T, Hq, Hkv, d, block_size,
                          topk, idx_w, status, sms, s));
@@ -421,6 +449,127 @@ int moba_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu
   return attn_fwd_impl(q, k, v, cu_dev, cu_host, nseq, Hq, Hkv, d, block_size, topk, scale,
                        block_idx_in, block_idx_out, o, lse, workspace, workspace_bytes, stream,
                        kPartialBudgetBytes);
+}
+
+int moba_attn_fwd_kconv(const void* q, const void* k, const void* v, const float* conv_w,
+                        int conv_width, const int32_t* cu_dev, const int32_t* cu_host, int nseq,
+                        int Hq, int Hkv, int d, int block_size, int topk, float scale,
+                        int32_t* block_idx_out, void* o, float* lse, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (!conv_w) return MOBA_ERR_ARG;
+  return attn_fwd_impl(q, k, v, cu_dev, cu_host, nseq, Hq, Hkv, d, block_size, topk, scale,
+                       nullptr, block_idx_out, o, lse, workspace, workspace_bytes, stream,
+                       kPartialBudgetBytes, conv_w, conv_width);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Host-side plan of a decode / chunked-prefill call: cache blocks and the query rows.
+struct DecodePlan {
+  int T = 0, Tq = 0, NB = 0, max_nb = 0;
+};
+
+int decode_plan(int nseq, const int32_t* cu, const int32_t* cuq, int Hq, int Hkv, int d, int B,
+                int topk, DecodePlan* P) {
+  int st = check_cu(nseq, cu);
+  if (st != MOBA_OK) return st;
+  if ((st = check_cu(nseq, cuq)) != MOBA_OK) return st;
+  if ((st = check_shape(Hq, Hkv, d, B, topk)) != MOBA_OK) return st;
+  for (int s = 0; s < nseq; ++s) {
+    const int L = cu[s + 1] - cu[s], n = cuq[s + 1] - cuq[s];
+    if (n > L) return MOBA_ERR_ARG;  // query rows are the newest tokens of the cache
+    const int nb = blocks_of(L, B);
+    if (nb > kMaxBlocksPerSeq) return MOBA_ERR_UNSUPPORTED;
+    P->max_nb = std::max(P->max_nb, nb);
+    P->NB += nb;
+  }
+  P->T = cu[nseq];
+  P->Tq = cuq[nseq];
+  if (static_cast<long long>(P->Tq) * Hq >= (1LL << 31) / 2) return MOBA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(P->T) * Hkv >= (1LL << 31) / 2) return MOBA_ERR_UNSUPPORTED;
+  return MOBA_OK;
+}
+
+struct DecodeLayout {
+  size_t status, blk_off, blk_seq, blk_start, blk_len, idx, part, total;
+};
+
+DecodeLayout decode_layout(const DecodePlan& P, int nseq, int Hq, int d, int B, int topk) {
+  DecodeLayout L;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t at = o; o = up256(o + bytes); return at; };
+  L.status = take(256);
+  L.blk_off = take(static_cast<size_t>(nseq + 1) * 4);
+  L.blk_seq = take(static_cast<size_t>(P.NB) * 4);
+  L.blk_start = take(static_cast<size_t>(P.NB) * 4);
+  L.blk_len = take(static_cast<size_t>(P.NB) * 4);
+  L.idx = take(static_cast<size_t>(Hq) * P.Tq * topk * 4);
+  L.part = take(static_cast<size_t>(P.Tq) * Hq * decode_parts(B, topk) * (d + 2) * 4);
+  L.total = o;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moba_decode_workspace_bytes(int nseq, const int32_t* cu_host, const int32_t* cuq_host,
+                                   int Hq, int Hkv, int d, int block_size, int topk) {
+  DecodePlan P;
+  if (decode_plan(nseq, cu_host, cuq_host, Hq, Hkv, d, block_size, topk, &P) != MOBA_OK) return 0;
+  return decode_layout(P, nseq, Hq, d, block_size, topk).total;
+}
+
+int moba_decode_fwd(const void* q, const void* k_cache, const void* v_cache,
+                    const float* centroids, const int32_t* cu_dev, const int32_t* cu_host,
+                    const int32_t* cuq_dev, const int32_t* cuq_host, int nseq, int Hq, int Hkv,
+                    int d, int block_size, int topk, float scale, const int32_t* block_idx_in,
+                    int32_t* block_idx_out, void* o, float* lse, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  DecodePlan P;
+  int st = decode_plan(nseq, cu_host, cuq_host, Hq, Hkv, d, block_size, topk, &P);
+  if (st != MOBA_OK) return st;
+  if (!(scale > 0.f) || scale > 1e30f) return MOBA_ERR_ARG;
+  if (P.Tq == 0) return MOBA_OK;
+  if (!q || !k_cache || !v_cache || !cu_dev || !cuq_dev || !o || !lse || !workspace)
+    return MOBA_ERR_ARG;
+  if (!block_idx_in && !centroids) return MOBA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      !aligned16(lse) || (centroids && !aligned16(centroids)))
+    return MOBA_ERR_ARG;
+  if ((block_idx_in && !aligned16(block_idx_in)) || (block_idx_out && !aligned16(block_idx_out)))
+    return MOBA_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOBA_ERR_ARG;
+  const DecodeLayout L = decode_layout(P, nseq, Hq, d, block_size, topk);
+  if (workspace_bytes < L.total) return MOBA_ERR_WORKSPACE;
+  int sms = 0;
+  if ((st = device_check(&sms)) != MOBA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  BlockTables tb;
+  tb.blk_off = at<int>(workspace, L.blk_off);
+  tb.blk_seq = at<int>(workspace, L.blk_seq);
+  tb.blk_start = at<int>(workspace, L.blk_start);
+  tb.blk_len = at<int>(workspace, L.blk_len);
+  int* status = at<int>(workspace, L.status);
+  MOBA_LAUNCH(kPlan, s, launch_plan(cu_dev, nseq, block_size, P.NB, tb, nullptr, 0, status, s));
+  int32_t* idx = block_idx_out ? block_idx_out : at<int32_t>(workspace, L.idx);
+  if (block_idx_in && idx != block_idx_in) {
+    if (cudaMemcpyAsync(idx, block_idx_in, static_cast<size_t>(Hq) * P.Tq * topk * 4,
+                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return MOBA_ERR_CUDA;
+  }
+  DecodeLaunch D;
+  D.q = q; D.k = k_cache; D.v = v_cache; D.cents = centroids;
+  D.cu = cu_dev; D.cuq = cuq_dev; D.blk_off = tb.blk_off;
+  D.idx = idx; D.idx_given = block_idx_in != nullptr;
+  D.part = at<float>(workspace, L.part);
+  D.o = o; D.lse = lse;
+  D.nseq = nseq; D.Tq = P.Tq; D.H = Hq; D.G = Hkv; D.d = d; D.B = block_size; D.topk = topk;
+  D.max_nb = P.max_nb; D.scale = scale;
+  MOBA_LAUNCH(kDecode, s, launch_decode(D, s));
+  return MOBA_OK;
 }
 
 int moba_device_status(const void* workspace, void* stream) {

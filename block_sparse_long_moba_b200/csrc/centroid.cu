@@ -18,10 +18,31 @@ namespace cg = cooperative_groups;
 
 namespace moba {
 
+// Short key convolution before pooling [FlashMoBA story: short convolutions within blocks].
+// With kconv[t] = sum_{m<W} w[m] k[t-m] inside the block (terms before the block's first key left
+// out), the block sum of the convolved keys follows from the plain block sum S and the block's
+// last W-1 keys, since key u contributes w[m] for every m with u + m still inside the block:
+//   sum_t kconv[t] = (sum_m w[m]) S - sum_{m=1}^{W-1} w[m] (k[e-1] + ... + k[e-m]),  e = block end
+// (the tail sum stops growing once it holds the whole block). `x` is the column in a token's row
+// of G * d keys, `last` points at column x of the block's last key, `ld` is the row stride.
+__device__ __forceinline__ float kconv_block_sum(float S, const float* __restrict__ cw, int W,
+                                                 int GD, int x, const __nv_bfloat16* last,
+                                                 size_t ld, int n) {
+  float wsum = 0.f;
+  for (int m = 0; m < W; ++m) wsum += __ldg(cw + static_cast<size_t>(m) * GD + x);
+  float res = wsum * S, tail = 0.f;
+  for (int m = 1; m < W; ++m) {
+    if (m <= n) tail += __bfloat162float(last[-static_cast<ptrdiff_t>((m - 1) * ld)]);
+    res = fmaf(-__ldg(cw + static_cast<size_t>(m) * GD + x), tail, res);
+  }
+  return res;
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) centroid_kernel(const __nv_bfloat16* __restrict__ k,
                                                        const int32_t* __restrict__ cu, int G,
-                                                       int B, int CL, float* __restrict__ out) {
+                                                       int B, int CL, float* __restrict__ out,
+                                                       const float* __restrict__ cw, int W) {
   constexpr int CPR = D / 8;     // 16-byte chunks per key row
   constexpr int RP = 256 / CPR;  // key rows covered by one pass of the CTA
   __shared__ float part[RP][D];
@@ -73,18 +94,26 @@ __global__ void __launch_bounds__(256) centroid_kernel(const __nv_bfloat16* __re
     red[threadIdx.x] = sum;
   }
   float* dst = out + (static_cast<size_t>(base + j) * G + g) * D;
+  auto finish = [&](float sum) -> float {
+    if (W > 0) {
+      const int x = g * D + threadIdx.x;
+      sum = kconv_block_sum(sum, cw, W, G * D, x,
+                            k + static_cast<size_t>(t0 + n - 1) * row_stride + x, row_stride, n);
+    }
+    return sum / static_cast<float>(n);
+  };
   if (CL > 1) {
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
     if (rank == 0 && threadIdx.x < D) {
       float sum = red[threadIdx.x];
       for (int q = 1; q < CL; ++q) sum += cluster.map_shared_rank(red, q)[threadIdx.x];
-      dst[threadIdx.x] = sum / static_cast<float>(n);
+      dst[threadIdx.x] = finish(sum);
     }
     cluster.sync();  // peers keep their shared memory alive until rank 0 has read it
   } else {
     __syncthreads();
-    if (threadIdx.x < D) dst[threadIdx.x] = red[threadIdx.x] / static_cast<float>(n);
+    if (threadIdx.x < D) dst[threadIdx.x] = finish(red[threadIdx.x]);
   }
 }
 
@@ -94,7 +123,8 @@ template <int NS>
 __global__ void __launch_bounds__(256) centroid_rows_kernel(const __nv_bfloat16* __restrict__ k,
                                                             const int32_t* __restrict__ cu,
                                                             int GD, int B, int CL,
-                                                            float* __restrict__ out) {
+                                                            float* __restrict__ out,
+                                                            const float* __restrict__ cw, int W) {
   extern __shared__ float sm_c[];  // NS == 1: [RPP][CPR][8] partial sums; then [CPR * 8] totals
   __shared__ int red_smem[32];
   const int rank = blockIdx.x % CL;
@@ -185,6 +215,12 @@ __global__ void __launch_bounds__(256) centroid_rows_kernel(const __nv_bfloat16*
   }
   float* dst = out + static_cast<size_t>(base + j) * GD;
   const float inv_n = 1.f / static_cast<float>(n);
+  auto finish = [&](float sum, int x) -> float {
+    if (W > 0)
+      sum = kconv_block_sum(sum, cw, W, GD, x, rowp + static_cast<size_t>(n - 1) * GD + x,
+                            static_cast<size_t>(GD), n);
+    return sum * inv_n;
+  };
   if (CL > 1) {
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
@@ -192,19 +228,20 @@ __global__ void __launch_bounds__(256) centroid_rows_kernel(const __nv_bfloat16*
       for (int x = tid; x < GD; x += 256) {
         float sum = sm_c[x];
         for (int q = 1; q < CL; ++q) sum += cluster.map_shared_rank(sm_c, q)[x];
-        dst[x] = sum * inv_n;
+        dst[x] = finish(sum, x);
       }
     }
     cluster.sync();  // peers keep their shared memory alive until rank 0 has read it
   } else {
     __syncthreads();
-    for (int x = tid; x < GD; x += 256) dst[x] = sm_c[x] * inv_n;
+    for (int x = tid; x < GD; x += 256) dst[x] = finish(sm_c[x], x);
   }
 }
 
 cudaError_t launch_centroids(const void* k, const int32_t* cu_dev, int nseq, int max_nb, int G,
                              int d, int B, int total_nb, int num_sms, float* out,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, const float* conv_w, int conv_width) {
+  const int W = conv_w ? conv_width : 0;
   const int GD = G * d;
   // whole rows need enough blocks to spread over the SMs (measured: 256 blocks of 4096 keys at
   // 91% of HBM, while 32 such blocks reached only a quarter of it in whole rows but half of it per
@@ -231,9 +268,11 @@ cudaError_t launch_centroids(const void* k, const int32_t* cu_dev, int nseq, int
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const __nv_bfloat16* kp = static_cast<const __nv_bfloat16*>(k);
-    if (NS == 1) return cudaLaunchKernelEx(&cfg, centroid_rows_kernel<1>, kp, cu_dev, GD, B, CL, out);
-    if (NS == 2) return cudaLaunchKernelEx(&cfg, centroid_rows_kernel<2>, kp, cu_dev, GD, B, CL, out);
-    return cudaLaunchKernelEx(&cfg, centroid_rows_kernel<4>, kp, cu_dev, GD, B, CL, out);
+    if (NS == 1)
+      return cudaLaunchKernelEx(&cfg, centroid_rows_kernel<1>, kp, cu_dev, GD, B, CL, out, conv_w, W);
+    if (NS == 2)
+      return cudaLaunchKernelEx(&cfg, centroid_rows_kernel<2>, kp, cu_dev, GD, B, CL, out, conv_w, W);
+    return cudaLaunchKernelEx(&cfg, centroid_rows_kernel<4>, kp, cu_dev, GD, B, CL, out, conv_w, W);
   }
   int CL = 1;
   while (CL < 8 && static_cast<long long>(total_nb) * G * CL < 8LL * num_sms) CL *= 2;
@@ -251,8 +290,9 @@ cudaError_t launch_centroids(const void* k, const int32_t* cu_dev, int nseq, int
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const __nv_bfloat16* kp = static_cast<const __nv_bfloat16*>(k);
-  if (d == 64) return cudaLaunchKernelEx(&cfg, centroid_kernel<64>, kp, cu_dev, G, B, CL, out);
-  return cudaLaunchKernelEx(&cfg, centroid_kernel<128>, kp, cu_dev, G, B, CL, out);
+  if (d == 64)
+    return cudaLaunchKernelEx(&cfg, centroid_kernel<64>, kp, cu_dev, G, B, CL, out, conv_w, W);
+  return cudaLaunchKernelEx(&cfg, centroid_kernel<128>, kp, cu_dev, G, B, CL, out, conv_w, W);
 }
 
 }  // namespace moba

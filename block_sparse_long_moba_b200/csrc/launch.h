@@ -10,9 +10,13 @@ namespace moba {
 cudaError_t launch_plan(const int32_t* cu_dev, int nseq, int B, int NB, const BlockTables& tb,
                         int* counts, int ncounts, int* status, cudaStream_t stream);
 
+// conv_w (nullable): weights [conv_width, G, d] fp32 of the short key convolution applied
+// inside each block before pooling.
+constexpr int kMaxKconvWidth = 16;
 cudaError_t launch_centroids(const void* k, const int32_t* cu_dev, int nseq, int max_nb, int G,
                              int d, int B, int total_nb, int num_sms, float* out,
-                             cudaStream_t stream);
+                             cudaStream_t stream, const float* conv_w = nullptr,
+                             int conv_width = 0);
 
 cudaError_t launch_gate(const void* q, const float* cents, const int32_t* cu_dev, int nseq,
                         int max_nb, int T, int H, int G, int d, int B, int topk, int32_t* idx,
@@ -87,13 +91,33 @@ cudaError_t launch_merge(const void* part_o, const float* part_lse, const int32_
                          int nseq, int T, int H, int d, int B, int topk, int T0, int ntok,
                          void* o, float* lse, cudaStream_t stream);
 
+// Decode / chunked prefill against a KV cache (csrc/decode.cu).
+struct DecodeLaunch {
+  const void* q;       // [Tq, H, d] bf16: the query rows (the last n_s tokens of each sequence)
+  const void* k;       // [T, G, d] bf16 cache
+  const void* v;
+  const float* cents;  // [NB, G, d] centroids of the cache's blocks
+  const int32_t* cu;   // [nseq + 1] cache lengths (device)
+  const int32_t* cuq;  // [nseq + 1] query rows per sequence (device)
+  const int* blk_off;  // [nseq + 1] first global block of each sequence (device)
+  int32_t* idx;        // [H, Tq, topk] routing (written by the gate unless idx_given)
+  bool idx_given;
+  float* part;         // [Tq, H, decode_parts] x (d + 2) fp32 partials
+  void* o;             // [Tq, H, d] bf16
+  float* lse;          // [H, Tq]
+  int nseq, Tq, H, G, d, B, topk, max_nb;
+  float scale;
+};
+int decode_parts(int B, int topk);
+cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream);
+
 // Whole forward pass on a caller-provided workspace (the body of moba_attn_fwd); the partial
 // outputs of one query chunk are kept under `partial_budget` bytes.
 int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu_dev,
                   const int32_t* cu_host, int nseq, int Hq, int Hkv, int d, int block_size,
                   int topk, float scale, const int32_t* block_idx_in, int32_t* block_idx_out,
                   void* o, float* lse, void* workspace, size_t workspace_bytes, void* stream,
-                  size_t partial_budget);
+                  size_t partial_budget, const float* conv_w = nullptr, int conv_width = 0);
 
 // Synchronises `stream`, reads the device status word at `word_dev` and maps it to a status.
 int read_status_word(const void* word_dev, void* stream);

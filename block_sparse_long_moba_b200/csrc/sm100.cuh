@@ -372,7 +372,8 @@ __device__ __forceinline__ void reg_fence(uint32_t& x) { asm volatile("" : "+r"(
 // 2^t on the FMA pipe, for t <= 8 (inputs below -120 are clamped; the result is then ~1e-36).
 // Round-to-nearest split t = n + f with |f| <= 1/2 (the 1.5 * 2^23 shifter), 2^f by a cubic fitted
 // here by iteratively reweighted least squares to minimise the relative error on [-1/2, 1/2]
-// (max relative error 2.2e-4, below the bf16 rounding of P), and 2^n added to the exponent bits.
+// (max relative error 2.21e-4 over [-120, 8], measured on the GPU against 2^t in double
+// precision; below the bf16 rounding of P), and 2^n added to the exponent bits.
 __device__ __forceinline__ float exp2_poly(float t) {
   t = fmaxf(t, -120.f);
   const float r = __fadd_rn(t, 12582912.f);

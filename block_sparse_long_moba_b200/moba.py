@@ -18,13 +18,15 @@ LIB_PATH = os.path.join(_HERE, "libmoba.so")
 STATUS = {0: "MOBA_OK", -1: "MOBA_ERR_ARG", -2: "MOBA_ERR_UNSUPPORTED", -3: "MOBA_ERR_WORKSPACE",
           -4: "MOBA_ERR_CUDA", -5: "MOBA_ERR_DEVICE_CHECK", -6: "MOBA_ERR_TIMEOUT"}
 KERNEL_CLASSES = ["centroid", "gate", "route_count", "route_scan", "route_scatter", "attention",
-                  "merge", "plan", "densify"]
+                  "merge", "plan", "densify", "decode"]
 
 # every symbol include/moba.h declares
 EXPORTS = ["moba_status_string", "moba_version", "moba_workspace_bytes", "moba_centroids",
            "moba_gate_topk", "moba_attn_fwd", "moba_device_status", "moba_timing_enable",
            "moba_timing_reset", "moba_timing_read", "moba_launch_count",
-           "moba_attn_fwd_noalloc", "moba_noalloc_status", "moba_set_wait_limit_ns"]
+           "moba_attn_fwd_noalloc", "moba_noalloc_status", "moba_set_wait_limit_ns",
+           "moba_centroids_kconv", "moba_attn_fwd_kconv", "moba_decode_workspace_bytes",
+           "moba_decode_fwd"]
 
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -69,6 +71,15 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moba_launch_count.restype = L
     lib.moba_attn_fwd_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P, P, P]
     lib.moba_attn_fwd_noalloc.restype = I
+    lib.moba_centroids_kconv.argtypes = [P, P, I, P, P, I, I, I, I, P, P]
+    lib.moba_centroids_kconv.restype = I
+    lib.moba_attn_fwd_kconv.argtypes = [P, P, P, P, I, P, P, I, I, I, I, I, I, F, P, P, P, P, S, P]
+    lib.moba_attn_fwd_kconv.restype = I
+    lib.moba_decode_workspace_bytes.argtypes = [I, P, P, I, I, I, I, I]
+    lib.moba_decode_workspace_bytes.restype = S
+    lib.moba_decode_fwd.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, P, P, S,
+                                    P]
+    lib.moba_decode_fwd.restype = I
     lib.moba_noalloc_status.argtypes = [P]
     lib.moba_noalloc_status.restype = I
     lib.moba_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
@@ -172,6 +183,31 @@ def moba_centroids(k: torch.Tensor, cu_seqlens: torch.Tensor, cu_seqlens_host, b
     return out
 
 
+def moba_centroids_kconv(k: torch.Tensor, conv_w: torch.Tensor, cu_seqlens: torch.Tensor,
+                         cu_seqlens_host, block_size: int, out: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """Centroids [NB, Hkv, d] fp32 of keys passed through the in-block short convolution with
+    weights conv_w [W, Hkv, d] fp32."""
+    what = "moba_centroids_kconv"
+    arr, nseq = _host_cu(cu_seqlens_host)
+    if not torch.is_tensor(k) or k.dim() != 3 or not torch.is_tensor(conv_w) or conv_w.dim() != 3:
+        _bad(what, "k must be [T, Hkv, d] and conv_w [W, Hkv, d]")
+    T, hkv, d = k.shape
+    _want(what, "k", k, torch.bfloat16, None, _ANY_DEVICE)
+    dev = _current_device(what, k)
+    _want(what, "conv_w", conv_w, torch.float32, (conv_w.shape[0], hkv, d), dev)
+    _want_cu(what, cu_seqlens, nseq, dev)
+    nb = num_blocks(list(arr), block_size)
+    if out is None:
+        out = torch.empty((nb, hkv, d), dtype=torch.float32, device=k.device)
+    _want(what, "out", out, torch.float32, (nb, hkv, d), dev)
+    st = load_library().moba_centroids_kconv(_ptr(k), _ptr(conv_w), conv_w.shape[0],
+                                             _ptr(cu_seqlens), arr, nseq, hkv, d, block_size,
+                                             _ptr(out), _stream(stream))
+    _check(st, what)
+    return out
+
+
 def moba_gate_topk(q: torch.Tensor, centroids: torch.Tensor, cu_seqlens: torch.Tensor,
                    cu_seqlens_host, block_size: int, topk: int,
                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
@@ -246,6 +282,113 @@ def moba_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens:
                            _ptr(block_idx_out), _ptr(o), _ptr(lse), _ptr(workspace),
                            ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check(st, "moba_attn_fwd")
+    return o, lse
+
+
+def moba_attn_fwd_kconv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                        conv_w: torch.Tensor, cu_seqlens: torch.Tensor, cu_seqlens_host,
+                        block_size: int, topk: int, scale: Optional[float] = None,
+                        block_idx_out: Optional[torch.Tensor] = None,
+                        o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None):
+    """MoBA forward with the routing computed on short-convolved keys (conv_w [W, Hkv, d] fp32);
+    returns (o, lse)."""
+    what = "moba_attn_fwd_kconv"
+    arr, nseq = _host_cu(cu_seqlens_host)
+    dev, T, hq, hkv, d = _check_qkv(what, q, k, v, cu_seqlens, nseq)
+    if not torch.is_tensor(conv_w) or conv_w.dim() != 3:
+        _bad(what, "conv_w must be [W, Hkv, d]")
+    _want(what, "conv_w", conv_w, torch.float32, (conv_w.shape[0], hkv, d), dev)
+    if scale is None:
+        scale = d ** -0.5
+    if block_idx_out is not None:
+        _want(what, "block_idx_out", block_idx_out, torch.int32, (hq, T, topk), dev)
+    lib = load_library()
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((hq, T), dtype=torch.float32, device=q.device)
+    _want(what, "o", o, torch.bfloat16, (T, hq, d), dev)
+    _want(what, "lse", lse, torch.float32, (hq, T), dev)
+    if workspace is None:
+        nbytes = int(lib.moba_workspace_bytes(nseq, arr, hq, hkv, d, block_size, topk))
+        if nbytes == 0 and T > 0:
+            raise MobaError(-1, "moba_workspace_bytes")
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    _want(what, "workspace", workspace, torch.uint8, None, dev)
+    st = lib.moba_attn_fwd_kconv(_ptr(q), _ptr(k), _ptr(v), _ptr(conv_w), conv_w.shape[0],
+                                 _ptr(cu_seqlens), arr, nseq, hq, hkv, d, block_size, topk,
+                                 ctypes.c_float(scale), _ptr(block_idx_out), _ptr(o), _ptr(lse),
+                                 _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+                                 _stream(stream))
+    _check(st, what)
+    return o, lse
+
+
+def moba_decode_workspace_bytes(cu_seqlens_host, cu_seqlens_q_host, hq: int, hkv: int, d: int,
+                                block_size: int, topk: int) -> int:
+    arr, nseq = _host_cu(cu_seqlens_host)
+    arq, nq = _host_cu(cu_seqlens_q_host)
+    if nq != nseq:
+        _bad("moba_decode_workspace_bytes", "cu_seqlens_q must have nseq + 1 entries")
+    return int(load_library().moba_decode_workspace_bytes(nseq, arr, arq, hq, hkv, d, block_size,
+                                                          topk))
+
+
+def moba_decode_fwd(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                    centroids: Optional[torch.Tensor], cu_seqlens: torch.Tensor, cu_seqlens_host,
+                    cu_seqlens_q: torch.Tensor, cu_seqlens_q_host, block_size: int, topk: int,
+                    scale: Optional[float] = None, block_idx_in: Optional[torch.Tensor] = None,
+                    block_idx_out: Optional[torch.Tensor] = None,
+                    o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None, stream=None):
+    """MoBA over the newest rows of a KV cache (decode: one row per sequence). q [Tq, Hq, d] are
+    the last n_s tokens of each sequence (cu_seqlens_q); returns (o [Tq, Hq, d], lse [Hq, Tq])."""
+    what = "moba_decode_fwd"
+    arr, nseq = _host_cu(cu_seqlens_host)
+    arq, nq = _host_cu(cu_seqlens_q_host)
+    if nq != nseq:
+        _bad(what, "cu_seqlens_q must have nseq + 1 entries")
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        if not torch.is_tensor(t) or t.dim() != 3:
+            _bad(what, f"{name} must be a 3-D tensor")
+    Tq, hq, d = q.shape
+    T, hkv = k_cache.shape[0], k_cache.shape[1]
+    _want(what, "q", q, torch.bfloat16, None, _ANY_DEVICE)
+    dev = _current_device(what, q)
+    _want(what, "k_cache", k_cache, torch.bfloat16, (T, hkv, d), dev)
+    _want(what, "v_cache", v_cache, torch.bfloat16, (T, hkv, d), dev)
+    _want_cu(what, cu_seqlens, nseq, dev)
+    _want(what, "cu_seqlens_q", cu_seqlens_q, torch.int32, (nseq + 1,), dev)
+    if centroids is not None:
+        _want(what, "centroids", centroids, torch.float32,
+              (num_blocks(list(arr), block_size), hkv, d), dev)
+    elif block_idx_in is None:
+        _bad(what, "centroids are required unless a routing is given")
+    for name, t in (("block_idx_in", block_idx_in), ("block_idx_out", block_idx_out)):
+        if t is not None:
+            _want(what, name, t, torch.int32, (hq, Tq, topk), dev)
+    if scale is None:
+        scale = d ** -0.5
+    lib = load_library()
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((hq, Tq), dtype=torch.float32, device=q.device)
+    _want(what, "o", o, torch.bfloat16, (Tq, hq, d), dev)
+    _want(what, "lse", lse, torch.float32, (hq, Tq), dev)
+    if workspace is None:
+        nbytes = int(lib.moba_decode_workspace_bytes(nseq, arr, arq, hq, hkv, d, block_size, topk))
+        if nbytes == 0 and Tq > 0:
+            raise MobaError(-1, "moba_decode_workspace_bytes")
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    _want(what, "workspace", workspace, torch.uint8, None, dev)
+    st = lib.moba_decode_fwd(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(centroids),
+                             _ptr(cu_seqlens), arr, _ptr(cu_seqlens_q), arq, nseq, hq, hkv, d,
+                             block_size, topk, ctypes.c_float(scale), _ptr(block_idx_in),
+                             _ptr(block_idx_out), _ptr(o), _ptr(lse), _ptr(workspace),
+                             ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check(st, what)
     return o, lse
 
 

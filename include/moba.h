@@ -86,6 +86,22 @@ int moba_centroids(const void* k, const int32_t* cu_seqlens_dev, const int32_t* 
                    int nseq, int Hkv, int d, int block_size, float* centroids, void* stream);
 
 /*
+ * Step 1 with a short key convolution before pooling [FlashMoBA story: short convolutions inside
+ * blocks cluster related keys and raise the routing signal]. The keys of every block first pass
+ * through a depthwise causal convolution of width W that never reaches into another block:
+ *   kconv[t, g, :] = sum_{m=0}^{W-1} conv_w[m, g, :] * k[t - m, g, :]   (terms with t - m before
+ *                    the block's first key left out),
+ * and the centroid is the mean of kconv over the block. Linear, no bias or activation (the pages
+ * give no kernel width, weights or activation). Only the routing sees the convolved keys;
+ * attention reads k as given.
+ * conv_w: device fp32 [W, Hkv, d], 16-byte aligned, 1 <= W <= 16 (MOBA_ERR_UNSUPPORTED above);
+ * the other arguments as for moba_centroids. Costs K's single pass plus W - 1 key rows per block.
+ */
+int moba_centroids_kconv(const void* k, const float* conv_w, int conv_width,
+                         const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host, int nseq,
+                         int Hkv, int d, int block_size, float* centroids, void* stream);
+
+/*
  * Step 2 — parameter-less causal top-k gate [MoBA paper summary, "Approach"; MoBA README,
  * "Parameter-less Gating Mechanism"].
  *   For query t in local block i of its sequence and head h (kv head g = h / (Hq/Hkv)):
@@ -122,6 +138,51 @@ int moba_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu
                   int block_size, int topk, float scale, const int32_t* block_idx_in,
                   int32_t* block_idx_out, void* o, float* lse, void* workspace,
                   size_t workspace_bytes, void* stream);
+
+/*
+ * moba_attn_fwd whose routing is computed on short-convolved keys (see moba_centroids_kconv):
+ * the same forward pass, with the centroids pooled from the convolved keys. There is no routing
+ * input (a given routing makes the convolution irrelevant); the workspace is sized by
+ * moba_workspace_bytes as for moba_attn_fwd.
+ */
+int moba_attn_fwd_kconv(const void* q, const void* k, const void* v, const float* conv_w,
+                        int conv_width, const int32_t* cu_seqlens_dev,
+                        const int32_t* cu_seqlens_host, int nseq, int Hq, int Hkv, int d,
+                        int block_size, int topk, float scale, int32_t* block_idx_out, void* o,
+                        float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * MoBA decode and chunked prefill against a KV cache [MoBA paper summary, "Approach" for the
+ * routing; its "Limitations": the paper's generation fell back to full attention, this applies
+ * the same block routing to the newest rows of a cache].
+ *   The cache holds nseq packed sequences: k_cache, v_cache bf16 [T, Hkv, d] with cu_seqlens as in
+ *   moba_attn_fwd (sequence s has L_s = cu[s+1] - cu[s] cached tokens, the new ones included).
+ *   Query rows: cu_seqlens_q [nseq + 1] (cuq[0] = 0, non-decreasing) gives n_s = cuq[s+1] - cuq[s]
+ *   <= L_s rows per sequence, which are its last n_s tokens (decode: n_s = 1). q bf16 [Tq, Hq, d]
+ *   with Tq = cuq[nseq]; row r of sequence s sits at position L_s - n_s + (r - cuq[s]).
+ *   Each row gets exactly the result moba_attn_fwd would give that token over its whole
+ *   sequence: the gate scores the past blocks j < i of its own position with the cached
+ *   centroids (fp32 [NB, Hkv, d], e.g. from moba_centroids on k_cache; only past blocks, which
+ *   are complete, are read, so a block's centroid needs computing once, when it completes), keeps
+ *   the current block and the top-(topk-1) past blocks, and attends their keys up to its own
+ *   position.
+ * block_idx_in : nullable [Hq, Tq, topk] routing to use instead of the gate (same contract as
+ *                moba_attn_fwd's; centroids may then be NULL).
+ * block_idx_out: nullable [Hq, Tq, topk], receives the routing used.
+ * o: bf16 [Tq, Hq, d]; lse: fp32 [Hq, Tq] (a sequence with no cached key gives o = 0, lse = -inf).
+ * workspace: at least moba_decode_workspace_bytes(...) bytes, 256-byte aligned.
+ * The path is HBM-bound: each (row, head) reads the K and V rows of its selected blocks once.
+ */
+size_t moba_decode_workspace_bytes(int nseq, const int32_t* cu_seqlens_host,
+                                   const int32_t* cu_seqlens_q_host, int Hq, int Hkv, int d,
+                                   int block_size, int topk);
+int moba_decode_fwd(const void* q, const void* k_cache, const void* v_cache,
+                    const float* centroids, const int32_t* cu_seqlens_dev,
+                    const int32_t* cu_seqlens_host, const int32_t* cu_seqlens_q_dev,
+                    const int32_t* cu_seqlens_q_host, int nseq, int Hq, int Hkv, int d,
+                    int block_size, int topk, float scale, const int32_t* block_idx_in,
+                    int32_t* block_idx_out, void* o, float* lse, void* workspace,
+                    size_t workspace_bytes, void* stream);
 
 /*
  * moba_attn_fwd for callers that cannot allocate device memory. The paper has no counterpart:
@@ -185,7 +246,8 @@ unsigned long long moba_set_wait_limit_ns(unsigned long long ns);
  * recorded events and writes, for each kernel class, the summed device milliseconds and launch
  * count since the last reset; kernel classes, in order: centroid, gate, route_count, route_scan,
  * route_scatter, attention, merge, plan, densify (d = 64: the routed query rows copied into one
- * dense array). Returns the number of classes (9), or a negative status.
+ * dense array), decode (moba_decode_fwd's kernels). Returns the number of classes (10), or a
+ * negative status.
  */
 int moba_timing_enable(int enable);
 int moba_timing_reset(void);

@@ -106,6 +106,36 @@ def centroids(k, cu_seqlens, block_size) -> np.ndarray:
     return out
 
 
+def key_conv(k, conv_w, cu_seqlens, block_size) -> np.ndarray:
+    """Short depthwise causal convolution of the keys inside each block, per kv head and channel:
+
+      kconv[t, g, :] = sum_{m=0}^{W-1} w[m, g, :] * k[t - m, g, :],  terms with t - m before the
+      first key of t's block left out (the convolution never reaches into another block).
+
+    [FlashMoBA story: short convolutions applied within blocks cluster related keys and raise the
+    routing signal.] The pages give no kernel width, weights or activation; the plainest reading
+    is a linear depthwise convolution with given weights w [W, Hkv, d], no bias or activation.
+    Returns [T, Hkv, d] fp64."""
+    kf = to_f64(k)
+    w = to_f64(conv_w)
+    W = w.shape[0]
+    bt = block_table(cu_seqlens, block_size)
+    out = np.zeros_like(kf)
+    for b in range(bt.num_blocks):
+        st, en = int(bt.start[b]), int(bt.end[b])
+        for t in range(st, en):
+            for m in range(W):
+                if t - m >= st:
+                    out[t] += w[m] * kf[t - m]
+    return out
+
+
+def centroids_kconv(k, conv_w, cu_seqlens, block_size) -> np.ndarray:
+    """Centroids of the convolved keys: the mean over each block of key_conv(...) [FlashMoBA story:
+    the short convolution is applied before the keys are pooled]. Returns [NB, Hkv, d] fp64."""
+    return centroids(key_conv(k, conv_w, cu_seqlens, block_size), cu_seqlens, block_size)
+
+
 @dataclass
 class Routing:
     """Block selection for a set of query tokens (all heads)."""
@@ -238,11 +268,49 @@ def attention(q, k, v, cu_seqlens, block_size, idx, scale, tokens) -> tuple:
     return out, lse
 
 
-def forward(q, k, v, cu_seqlens, block_size, topk, scale, tokens=None):
-    """Whole path: centroids -> gate -> attention. Returns (routing, O [n,H,d], LSE [H,n])."""
-    cents = centroids(k, cu_seqlens, block_size)
+def forward(q, k, v, cu_seqlens, block_size, topk, scale, tokens=None, conv_w=None):
+    """Whole path: centroids -> gate -> attention. Returns (routing, O [n,H,d], LSE [H,n]).
+    With conv_w the centroids pool the convolved keys (key_conv); attention reads the keys as
+    given: the convolution only shapes the routing."""
+    cents = (centroids(k, cu_seqlens, block_size) if conv_w is None
+             else centroids_kconv(k, conv_w, cu_seqlens, block_size))
     rt = select_blocks(q, cents, cu_seqlens, block_size, topk, tokens)
     out, lse = attention(q, k, v, cu_seqlens, block_size, rt.idx, scale, rt.tokens)
+    return rt, out, lse
+
+
+def cache_row_positions(cu_seqlens, cu_seqlens_q) -> np.ndarray:
+    """Absolute positions of query rows that are the last n_s tokens of each cached sequence:
+    row r of sequence s sits at cu[s] + L_s - n_s + (r - cuq[s])."""
+    cu = [int(x) for x in cu_seqlens]
+    cuq = [int(x) for x in cu_seqlens_q]
+    pos = []
+    for s in range(len(cu) - 1):
+        L, n = cu[s + 1] - cu[s], cuq[s + 1] - cuq[s]
+        assert 0 <= n <= L
+        pos += [cu[s] + L - n + x for x in range(n)]
+    return np.asarray(pos, np.int64)
+
+
+def decode(q_rows, k, v, cu_seqlens, cu_seqlens_q, block_size, topk, scale, cents=None):
+    """MoBA over the newest rows of a KV cache (decode: one row per sequence).
+
+    The rows are the last n_s tokens of each sequence, and each gets exactly what the prefill
+    forward pass gives that token over its whole sequence: the same gate on the past blocks of its
+    own position, the same attention up to its own position [MoBA paper summary, "Approach"; its
+    "Limitations" note the paper decoded with full attention, so decode-time routing is the
+    plainest reading: the prefill rule applied to the newest token]. cents: the cache's centroids
+    (computed from k when None). Returns (Routing, O [Tq,H,d], LSE [H,Tq]).
+    """
+    tokens = cache_row_positions(cu_seqlens, cu_seqlens_q)
+    qr = to_f64(q_rows)
+    T = int(k.shape[0])
+    q_full = np.zeros((T,) + qr.shape[1:])
+    q_full[tokens] = qr
+    if cents is None:
+        cents = centroids(k, cu_seqlens, block_size)
+    rt = select_blocks(q_full, cents, cu_seqlens, block_size, topk, tokens)
+    out, lse = attention(q_full, k, v, cu_seqlens, block_size, rt.idx, scale, tokens)
     return rt, out, lse
 
 

@@ -94,14 +94,29 @@ def test_centroids_and_gate_host_side_errors(lib):
     assert lib.moba_gate_topk(FAKE, FAKE, FAKE, _cu([0, 0]), 1, 2, 2, 64, 128, 3, FAKE, None) == 0
 
 
+def test_kconv_host_side_errors(lib):
+    cu = _cu([0, 1024])
+    kc = lib.moba_centroids_kconv
+    assert kc(FAKE, None, 3, FAKE, cu, 1, 2, 64, 128, FAKE, None) == -1        # no weights
+    assert kc(FAKE, FAKE, 0, FAKE, cu, 1, 2, 64, 128, FAKE, None) == -1        # width 0
+    assert kc(FAKE, FAKE, 17, FAKE, cu, 1, 2, 64, 128, FAKE, None) == -2       # width > 16
+    assert kc(FAKE, ctypes.c_void_p(0x100004), 3, FAKE, cu, 1, 2, 64, 128, FAKE, None) == -1
+    assert kc(FAKE, FAKE, 3, FAKE, _cu([0, 0]), 1, 2, 64, 128, FAKE, None) == 0  # empty input
+    af = lib.moba_attn_fwd_kconv
+    assert af(FAKE, FAKE, FAKE, None, 3, FAKE, cu, 1, 2, 2, 64, 128, 3, ctypes.c_float(0.1),
+              None, FAKE, FAKE, FAKE, ctypes.c_size_t(1 << 40), None) == -1
+    assert af(FAKE, FAKE, FAKE, FAKE, 17, FAKE, cu, 1, 2, 2, 64, 128, 3, ctypes.c_float(0.1),
+              None, FAKE, FAKE, FAKE, ctypes.c_size_t(1 << 40), None) == -2
+
+
 def test_timing_classes_match_the_binding(lib):
     """moba_timing_read reports one entry per kernel class, in the binding's order (no GPU: with
     timing off nothing is recorded and no event is touched)."""
     from block_sparse_long_moba_b200 import moba
     assert lib.moba_timing_reset() == 0
     n = lib.moba_timing_read(None, None, 0)
-    assert n == len(moba.KERNEL_CLASSES) == 9
-    assert moba.KERNEL_CLASSES[-1] == "densify"
+    assert n == len(moba.KERNEL_CLASSES) == 10
+    assert moba.KERNEL_CLASSES[-2:] == ["densify", "decode"]
 
 
 @pytest.mark.parametrize("value,was_on", [("1", "1"), ("0", "0"), (None, "0")])

@@ -4,11 +4,14 @@ import pytest
 
 from oracle import moba_ref as ref
 from tests import test_oracle as pins
+from tests import test_oracle_decode as dpins
+from tests import test_oracle_kconv as kpins
 
 _orig_centroids = ref.centroids
 _orig_select = ref.select_blocks
 _orig_attention = ref.attention
 _orig_gate_scores = ref.gate_scores
+_orig_key_conv = ref.key_conv
 
 
 def _sum_not_mean(k, cu, B):
@@ -86,6 +89,28 @@ def _magnitude_of_the_sum(q, cents, cu, B, topk, tokens=None):
     return rt
 
 
+def _conv_across_blocks(k, conv_w, cu, B):
+    # the convolution reaches back into the previous block (one long sequence per cu segment)
+    return _orig_key_conv(k, conv_w, cu, 10 ** 9)
+
+
+def _conv_anticausal(k, conv_w, cu, B):
+    # the kernel applied to later keys (t + m) instead of earlier ones
+    kf = ref.to_f64(k)[::-1].copy()
+    T = kf.shape[0]
+    bt = ref.block_table(cu, B)
+    rev_cu = [0] + [T - int(x) for x in bt.start[::-1]]
+    out = _orig_key_conv(kf, conv_w, rev_cu, 10 ** 9)
+    return out[::-1].copy()
+
+
+def _rows_at_the_front(cu, cuq):
+    # query rows taken as the first n_s tokens of each sequence instead of the last
+    cu, cuq = [int(x) for x in cu], [int(x) for x in cuq]
+    return np.asarray([cu[s] + x for s in range(len(cu) - 1) for x in range(cuq[s + 1] - cuq[s])],
+                      np.int64)
+
+
 @pytest.mark.parametrize("target,fake,pin", [
     ("centroids", _sum_not_mean, pins.test_centroid_closed_form_with_ragged_tail),
     ("select_blocks", _negated_gate, pins.test_gate_constructed_case),
@@ -94,6 +119,9 @@ def _magnitude_of_the_sum(q, cents, cu, B, topk, tokens=None):
     ("select_blocks", _margin_off_by_one, pins.test_gate_margin_and_boundary_hand_derived),
     ("gate_scores", _gate_scores_gqa_modulo, pins.test_gate_scores_hand_derived_gqa),
     ("select_blocks", _magnitude_of_the_sum, pins.test_gate_magnitude_sums_absolute_terms),
+    ("key_conv", _conv_across_blocks, kpins.test_convolution_stops_at_the_block_start),
+    ("key_conv", _conv_anticausal, kpins.test_pure_delay_closed_form),
+    ("cache_row_positions", _rows_at_the_front, dpins.test_row_positions),
 ])
 def test_pin_catches_planted_mistake(monkeypatch, target, fake, pin):
     monkeypatch.setattr(ref, target, fake)
