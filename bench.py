@@ -513,6 +513,138 @@ def summarize(w: wl.Workload, m: dict, steps: int, world: int, peaks: dict) -> d
     }
 
 
+def measure_backward(w: wl.Workload, steps: int, warmup: int, peaks: dict) -> dict:
+    """Times moba_attn_bwd on `w` (one GPU): the forward pass runs once first for O, LSE and the
+    routing; dO is seeded N(0, 1). Useful FLOPs: 10 d per attended (query, key) pair and head
+    (S recomputed, dP, dV, dK, dQ); the key-stationary kernel issues 8 d of them per pair (S, dP,
+    dV, dK) and the query-stationary one 6 d (S, dP, dQ)."""
+    from block_sparse_long_moba_b200 import moba
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v, cu = wl.make_inputs(w, seed=0, device=dev)
+    T, H, d = w.total_tokens, w.hq, w.d
+    idx = torch.empty((H, T, w.topk), dtype=torch.int32, device=dev)
+    o, lse = moba.moba_attn_fwd(q, k, v, cu, w.cu_seqlens, w.block_size, w.topk, w.scale,
+                                block_idx_out=idx)
+    g = torch.Generator(device=dev).manual_seed(5)
+    d_o = torch.randn(q.shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(moba.moba_bwd_workspace_bytes(w.cu_seqlens, H, w.hkv, d, w.block_size,
+                                                   w.topk), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        moba.moba_attn_bwd(q, k, v, o, lse, d_o, idx, cu, w.cu_seqlens, w.block_size, w.topk,
+                           w.scale, dq=dq, dk=dk, dv=dv, workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if moba.moba_device_status(ws) != 0:
+        raise RuntimeError(f"{w.name} backward: device status after warm-up")
+    moba.timing_reset()
+    moba.timing_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    moba.timing_enable(False)
+    per = moba.timing_read()
+    ms = ev0.elapsed_time(ev1) / steps
+    if moba.moba_device_status(ws) != 0:
+        raise RuntimeError(f"{w.name} backward: device status after the timed region")
+    pairs = attended_pairs(w)
+    peak = peaks["bf16_tflops_sustained"]
+    kern = {}
+    for name, flop_per_pair in (("bwd_dkdv", 8.0 * d), ("bwd_dq", 6.0 * d), ("bwd_aux", None)):
+        kms, kn = per.get(name, (0.0, 0))
+        if kn == 0:
+            continue
+        ent = {"ms_per_step": kms / steps, "launches_per_step": kn / steps}
+        if flop_per_pair:
+            tf = flop_per_pair * pairs / (kms / steps / 1e3) / 1e12
+            ent.update({"tflops": tf, "frac": tf / peak})
+        kern[name] = ent
+    for name in ("route_count", "route_scan", "route_scatter", "plan"):
+        kms, kn = per.get(name, (0.0, 0))
+        if kn:
+            kern[name] = {"ms_per_step": kms / steps}
+    useful = 10.0 * d * pairs
+    return {"workload": w.name, "steps": steps, "warmup": warmup, "ms_per_step": ms,
+            "tflops_useful": useful / (ms / 1e3) / 1e12,
+            "frac_of_peak_sustained": useful / (ms / 1e3) / 1e12 / peak,
+            "useful_tflop": useful / 1e12, "kernels": kern,
+            "peak": peak, "peak_kind": f"bf16 dense sustained, {peaks['source']}"}
+
+
+DECODE_CACHE = dict(nseq=8, L=131072, hq=32, hkv=8, d=128, block_size=4096, topk=12)
+
+
+def measure_decode(steps: int, warmup: int, peaks: dict) -> dict:
+    """Times moba_decode_fwd: one new query per sequence for 8 sequences with 128K cached tokens
+    each (the Llama-3.1-8B attention shape). Algorithmic bytes: the K and V rows of the blocks the
+    query heads of a kv group select (their union, read once), plus Q, the past centroids and the
+    outputs; the kernels read each head's blocks separately, so the union is the floor that L2
+    reuse across a group's heads can reach."""
+    from block_sparse_long_moba_b200 import moba
+
+    c = DECODE_CACHE
+    cu_l = [c["L"] * s for s in range(c["nseq"] + 1)]
+    w = wl.custom(cu_l, c["hq"], c["hkv"], c["d"], c["block_size"], c["topk"], "offset",
+                  name="decode_128k_b8")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q_all, k, v, cu = wl.make_inputs(w, seed=0, device=dev)
+    last = torch.tensor([x - 1 for x in cu_l[1:]], device=dev)
+    q = q_all[last].contiguous()
+    del q_all
+    cuq_l = list(range(c["nseq"] + 1))
+    cuq = torch.tensor(cuq_l, dtype=torch.int32, device=dev)
+    cents = moba.moba_centroids(k, cu, cu_l, c["block_size"])
+    H, d, nq = c["hq"], c["d"], c["nseq"]
+    idx = torch.empty((H, nq, c["topk"]), dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((H, nq), dtype=torch.float32, device=dev)
+    ws = torch.empty(moba.moba_decode_workspace_bytes(cu_l, cuq_l, H, c["hkv"], d,
+                                                      c["block_size"], c["topk"]),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        moba.moba_decode_fwd(q, k, v, cents, cu, cu_l, cuq, cuq_l, c["block_size"], c["topk"],
+                             w.scale, block_idx_out=idx, o=o, lse=lse, workspace=ws,
+                             stream=stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / steps
+    # union of the blocks selected by the heads of each (row, kv group); every block is full
+    r = H // c["hkv"]
+    sel = idx.view(c["hkv"], r, nq, c["topk"]).permute(0, 2, 1, 3).reshape(c["hkv"], nq, -1)
+    uniq = sum(len(set(x for x in row.tolist() if x >= 0)) for grp in sel for row in grp)
+    kv_bytes = uniq * c["block_size"] * d * 2 * 2
+    nb_past = c["L"] // c["block_size"] - 1
+    other = nq * H * d * 2 * 2 + nq * H * nb_past * d * 4 + nq * H * 4
+    per_head = nq * H * c["topk"] * c["block_size"] * d * 2 * 2
+    gbs = (kv_bytes + other) / (ms / 1e3) / 1e9
+    return {"workload": w.name, "steps": steps, "warmup": warmup,
+            "config": {"nseq": nq, "cache_tokens_per_seq": c["L"], "rows_per_seq": 1, "hq": H,
+                       "hkv": c["hkv"], "d": d, "block_size": c["block_size"],
+                       "topk": c["topk"]},
+            "ms_per_step": ms, "rows_per_s": nq / (ms / 1e3),
+            "bytes_algorithmic": kv_bytes + other, "bytes_per_head_reads": per_head + other,
+            "gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"]}
+
+
 def run_ours(args):
     from block_sparse_long_moba_b200 import build, moba
 
@@ -550,6 +682,13 @@ def run_ours(args):
             del mx
             torch.cuda.empty_cache()
 
+    bwd = dec = None
+    if world == 1 and not args.no_extra:
+        bwd = measure_backward(w, 3, 2, peaks)
+        torch.cuda.empty_cache()
+        dec = measure_decode(20, 3, peaks)
+        torch.cuda.empty_cache()
+
     if rank == 0:
         ms_step = summ["ms_per_step"]
         att = summ["attention"]
@@ -584,6 +723,10 @@ def run_ours(args):
         }
         if extra:
             line["workloads"] = extra
+        if bwd:
+            line["backward"] = bwd
+        if dec:
+            line["decode"] = dec
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)

@@ -20,15 +20,18 @@ using namespace moba;
 namespace {
 
 constexpr size_t kPartialBudgetBytes = 16ull << 30;  // per-chunk partial outputs + routing lists
-constexpr int kNumClasses = 10;
+constexpr int kNumClasses = 13;
 enum KernelClass {
   kCentroid = 0, kGate, kRouteCount, kRouteScan, kRouteScatter, kAttn, kMerge, kPlan, kDensify,
-  kDecode
+  kDecode, kBwdDkdv, kBwdDq, kBwdAux
 };
 
 std::atomic<long long> g_launches{0};
 // Limit of one pipeline wait inside the attention kernel (0 = the built-in 2 s).
 std::atomic<unsigned long long> g_wait_limit_ns{0};
+// Diagnostics: when set, the attention kernel's MMA issuer first waits on a barrier that nothing
+// arrives on, so that the wait runs out and every CTA takes its abort path.
+std::atomic<int> g_diag_stall{0};
 
 // ------------------------------------------------------------------------------- timing hooks
 // Timing starts enabled when the process sets MOBA_TIMING=1.
@@ -57,7 +60,8 @@ Timing& timing() { static Timing t; return t; }
 const char* const kClassNames[kNumClasses] = {"moba_centroids", "moba_gate", "moba_route_count",
                                                "moba_route_scan", "moba_route_scatter",
                                                "moba_attention", "moba_merge", "moba_plan",
-                                               "moba_densify", "moba_decode"};
+                                               "moba_densify", "moba_decode",
+                                               "moba_bwd_dkdv", "moba_bwd_dq", "moba_bwd_aux"};
 
 // Brackets one kernel launch: an NVTX range named for its class (seen by profilers; a no-op
 // otherwise) and, when timing is enabled, CUDA events on the launching stream.
@@ -406,6 +410,7 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu
     A.T = P.T; A.H = Hq; A.G = Hkv; A.d = d; A.B = block_size; A.topk = topk; A.NB = P.NB;
     A.b0 = c.b0; A.nblk = c.nblk; A.T0 = c.T0; A.scale = scale;
     A.wait_ns = g_wait_limit_ns.load();
+    A.diag_stall = g_diag_stall.load();
     const long long P256 = (block_size + kItemRows - 1) / kItemRows;
     const long long items = static_cast<long long>(P.max_tiles) + P256 * c.nblk * Hq;
     A.grid = static_cast<int>(std::min<long long>(sms, items));
@@ -572,6 +577,116 @@ int moba_decode_fwd(const void* q, const void* k_cache, const void* v_cache,
   return MOBA_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+struct BwdLayout {
+  size_t status, blk_off, blk_seq, blk_start, blk_len, counts, cursor, tiles, entries, dsum, dq_acc,
+      total;
+};
+
+BwdLayout bwd_layout(const Plan& P, int nseq, int Hq, int Hkv, int d, int topk) {
+  BwdLayout L;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t at = o; o = up256(o + bytes); return at; };
+  const size_t rows = static_cast<size_t>(P.T) * Hq;
+  const size_t ent = rows * (topk - 1);
+  L.status = take(256);
+  L.blk_off = take(static_cast<size_t>(nseq + 1) * 4);
+  L.blk_seq = take(static_cast<size_t>(P.NB) * 4);
+  L.blk_start = take(static_cast<size_t>(P.NB) * 4);
+  L.blk_len = take(static_cast<size_t>(P.NB) * 4);
+  L.counts = take(static_cast<size_t>(Hkv) * P.NB * 4);
+  L.cursor = take(static_cast<size_t>(Hkv) * P.NB * 4);
+  L.tiles = take((ent / kItemRows + static_cast<size_t>(Hkv) * P.NB + 1) * 16);
+  L.entries = take(std::max<size_t>(ent, 1) * 4);
+  L.dsum = take(rows * 4);
+  L.dq_acc = take(rows * d * 4);
+  L.total = o;
+  return L;
+}
+
+int bwd_check(int nseq, const int32_t* cu_host, int Hq, int Hkv, int d, int B, int topk, Plan* P) {
+  int st = check_cu(nseq, cu_host);
+  if (st != MOBA_OK) return st;
+  if ((st = check_shape(Hq, Hkv, d, B, topk)) != MOBA_OK) return st;
+  // one query chunk over the whole problem: the routing lists of every row at once
+  if ((st = make_plan(nseq, cu_host, Hq, Hkv, d, B, topk, P, ~static_cast<size_t>(0) >> 1)) !=
+      MOBA_OK)
+    return st;
+  if (static_cast<long long>(P->T) * Hq * topk >= (1LL << 31)) return MOBA_ERR_UNSUPPORTED;
+  return MOBA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moba_bwd_workspace_bytes(int nseq, const int32_t* cu_seqlens_host, int Hq, int Hkv, int d,
+                                int block_size, int topk) {
+  Plan P;
+  if (bwd_check(nseq, cu_seqlens_host, Hq, Hkv, d, block_size, topk, &P) != MOBA_OK) return 0;
+  return bwd_layout(P, nseq, Hq, Hkv, d, topk).total;
+}
+
+int moba_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                  const void* d_o, const int32_t* block_idx, const int32_t* cu_dev,
+                  const int32_t* cu_host, int nseq, int Hq, int Hkv, int d, int block_size,
+                  int topk, float scale, void* dq, void* dk, void* dv, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  Plan P;
+  int st = bwd_check(nseq, cu_host, Hq, Hkv, d, block_size, topk, &P);
+  if (st != MOBA_OK) return st;
+  if (!(scale > 0.f) || scale > 1e30f) return MOBA_ERR_ARG;
+  if (P.T == 0) return MOBA_OK;
+  const void* ptrs[] = {q, k, v, o, lse, d_o, block_idx, dq, dk, dv};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return MOBA_ERR_ARG;
+  if (!cu_dev || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return MOBA_ERR_ARG;
+  const BwdLayout L = bwd_layout(P, nseq, Hq, Hkv, d, topk);
+  if (workspace_bytes < L.total) return MOBA_ERR_WORKSPACE;
+  int sms = 0;
+  if ((st = device_check(&sms)) != MOBA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  BlockTables tb;
+  tb.blk_off = at<int>(workspace, L.blk_off);
+  tb.blk_seq = at<int>(workspace, L.blk_seq);
+  tb.blk_start = at<int>(workspace, L.blk_start);
+  tb.blk_len = at<int>(workspace, L.blk_len);
+  int* status = at<int>(workspace, L.status);
+  int* n_tiles = status + 1;
+  int* counts = at<int>(workspace, L.counts);
+  int* cursor = at<int>(workspace, L.cursor);
+  int4* tiles = at<int4>(workspace, L.tiles);
+  int* entries = at<int>(workspace, L.entries);
+  const int NBK = Hkv * P.NB;
+  MOBA_LAUNCH(kPlan, s, launch_plan(cu_dev, nseq, block_size, P.NB, tb, counts, NBK, status, s));
+  MOBA_LAUNCH(kRouteCount, s,
+              launch_route_count(block_idx, tb, P.T, Hq, Hkv, topk, P.NB, 0, P.NB, 0, P.max_nb,
+                                 counts, status, s));
+  MOBA_LAUNCH(kRouteScan, s, launch_route_scan(counts, NBK, cursor, tiles, n_tiles, s));
+  MOBA_LAUNCH(kRouteScatter, s,
+              launch_route_scatter(block_idx, tb, P.T, Hq, Hkv, topk, P.NB, 0, P.NB, 0, P.max_nb,
+                                   cursor, entries, s));
+  BwdLaunch B;
+  B.q = q; B.k = k; B.v = v; B.o = o; B.dout = d_o; B.lse = lse;
+  B.entries = entries; B.bucket_end = cursor; B.tiles = tiles; B.n_routed = n_tiles;
+  B.tb = tb;
+  B.dsum = at<float>(workspace, L.dsum);
+  B.dq_acc = at<float>(workspace, L.dq_acc);
+  B.dq = dq; B.dk = dk; B.dv = dv; B.status = status;
+  B.T = P.T; B.H = Hq; B.G = Hkv; B.d = d; B.B = block_size; B.topk = topk; B.NB = P.NB;
+  B.num_sms = sms; B.scale = scale;
+  B.wait_ns = g_wait_limit_ns.load();
+  MOBA_LAUNCH(kBwdAux, s, launch_bwd_pre(B, s));
+  MOBA_LAUNCH(kBwdDkdv, s, launch_bwd_dkdv(B, s));
+  MOBA_LAUNCH(kBwdDq, s, launch_bwd_dq(B, s));
+  MOBA_LAUNCH(kBwdAux, s, launch_bwd_finish(B, s));
+  return MOBA_OK;
+}
+
 int moba_device_status(const void* workspace, void* stream) {
   if (!workspace) return MOBA_ERR_ARG;
   return moba::read_status_word(workspace, stream);
@@ -581,6 +696,8 @@ unsigned long long moba_set_wait_limit_ns(unsigned long long ns) {
   const unsigned long long was = g_wait_limit_ns.exchange(ns);
   return was ? was : kWaitTimeoutNs;
 }
+
+int moba_set_diag_stall(int on) { return g_diag_stall.exchange(on != 0 ? 1 : 0); }
 
 int moba_timing_enable(int enable) {
   Timing& T = timing();

@@ -69,6 +69,7 @@ struct AttnArgs {
   int n_diag;              // P2 * nblk * H diagonal items (some may be empty)
   float scale_log2;        // scale * log2(e)
   unsigned long long wait_ns;  // limit of one pipeline wait (abort drains use kDrainTimeoutNs)
+  int diag_stall;              // diagnostics: the MMA issuer first waits on a barrier nobody arrives on
 };
 
 struct __align__(16) Item {
@@ -236,7 +237,7 @@ struct D64Bars {
   uint64_t q_full[D64Cfg::QB], q_empty[D64Cfg::QB];
   uint64_t k_full[D64Cfg::NK], k_empty[D64Cfg::NK], v_full[D64Cfg::NV], v_empty[D64Cfg::NV];
   uint64_t s_full[2], p_full[2], o_full[2][2];
-  uint64_t drain;
+  uint64_t drain, never;
   uint32_t tmem_base;
   int abort_flag;
   ItemRing ring;
@@ -286,6 +287,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->o_full[x][1], 1);
     }
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->never, 1);
     for (int x = 0; x < kRing; ++x) {
       mbar_init(&ring->full[x], 1);
       mbar_init(&ring->empty[x], C::RING_CONSUMERS);
@@ -399,7 +401,8 @@ __global__ void __launch_bounds__(384, 1)
       bool pend = false, pend_first = false, pend_last = false;
       int pend_sv = 0;
       uint32_t pend_c = 0, pend_item = 0;
-      for (uint32_t lt = 0;; ++lt) {
+      if (a.diag_stall) ok = wait(&bars->never, 0);  // runs out: the whole CTA takes its abort path
+      for (uint32_t lt = 0; ok; ++lt) {
         Item it;
         ok = __all_sync(0xffffffffu, pop(lt, it));
         if (!ok || it.kind < 0) break;
@@ -734,7 +737,7 @@ struct PvtBars {
   uint64_t k_full[2], k_empty[2], v_full, v_empty;
   uint64_t s_full[2], s_free[2];
   uint64_t p_full, pv_done;
-  uint64_t drain;
+  uint64_t drain, never;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -799,6 +802,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&bars->p_full, 256);
     mbar_init(&bars->pv_done, 1);
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->never, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -919,6 +923,7 @@ __global__ void __launch_bounds__(384, 1)
         return true;
       };
       uint32_t J = 0, lt = 0;
+      if (a.diag_stall) ok = wait(&bars->never, 0);  // runs out: the whole CTA takes its abort path
       for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
         const Item it = decode_item(a, w, n_routed);
         if (it.kind == 0) continue;
@@ -1203,12 +1208,8 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 // ---------------------------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-static EncodeTiledFn get_encode_fn() {
+EncodeTiledFn get_encode_fn() {
   static EncodeTiledFn fn = nullptr;
   if (!fn) {
     void* p = nullptr;
@@ -1222,7 +1223,7 @@ static EncodeTiledFn get_encode_fn() {
 }
 
 // [T, G, D] bf16 -> 3-D map (D, G, T), box (64, 1, 128), 128-byte swizzle, zero fill out of range.
-static bool make_kv_map(CUtensorMap* map, const void* base, int T, int G, int D) {
+bool make_kv_map(CUtensorMap* map, const void* base, int T, int G, int D) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(G),
@@ -1237,7 +1238,7 @@ static bool make_kv_map(CUtensorMap* map, const void* base, int T, int G, int D)
 
 // [T * H, D] bf16 query rows -> 2-D map (D, T * H), box (64, 1): one row per box, as the row
 // gather (tile::gather4) requires; 128-byte swizzle.
-static bool make_q_rows_map(CUtensorMap* map, const void* base, long long rows, int D) {
+bool make_q_rows_map(CUtensorMap* map, const void* base, long long rows, int D) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
@@ -1293,6 +1294,7 @@ cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream) {
   a.n_diag = a.P2 * L.nblk * L.H;
   a.scale_log2 = L.scale * 1.4426950408889634f;
   a.wait_ns = L.wait_ns > 0 ? L.wait_ns : kWaitTimeoutNs;
+  a.diag_stall = L.diag_stall;
   const int grid = L.grid > 0 ? L.grid : 1;
   // setmaxnreg.inc would wait forever if the launch had fewer registers than the split assumes
   {

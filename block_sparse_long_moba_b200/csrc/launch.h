@@ -1,6 +1,7 @@
 // Host-side launchers of the MoBA kernels (internal to libmoba.so).
 #pragma once
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -83,9 +84,21 @@ struct AttnLaunch {
   float scale;
   int grid;
   unsigned long long wait_ns = 0;  // pipeline-wait limit; 0 = kWaitTimeoutNs
+  int diag_stall = 0;              // diagnostics: make the MMA issuer's first wait run out
 };
 
 cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream);
+
+// TMA tensor maps (csrc/attn.cu): the driver's cuTensorMapEncodeTiled, a [T, G, D] bf16 key or
+// value tensor as a 3-D map (D, G, T) with a (64, 1, 128) box and the 128-byte swizzle, and
+// [rows, D] bf16 rows as a 2-D map with a one-row box (for tile::gather4), 128-byte swizzle.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_fn();
+bool make_kv_map(CUtensorMap* map, const void* base, int T, int G, int D);
+bool make_q_rows_map(CUtensorMap* map, const void* base, long long rows, int D);
 
 cudaError_t launch_merge(const void* part_o, const float* part_lse, const int32_t* cu_dev,
                          int nseq, int T, int H, int d, int B, int topk, int T0, int ntok,
@@ -110,6 +123,30 @@ struct DecodeLaunch {
 };
 int decode_parts(int B, int topk);
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream);
+
+// Backward pass of the routed attention (csrc/attn_bwd.cu).
+struct BwdLaunch {
+  const void *q, *k, *v, *o, *dout;  // bf16 [T, H or G, d]
+  const float* lse;                  // [H, T]
+  const int* entries;                // routed entries grouped by (g, b) (routing inversion)
+  const int* bucket_end;             // [G * NB] end of every list after the scatter
+  const int4* tiles;                 // routed 256-row items
+  const int* n_routed;
+  BlockTables tb;
+  float* dsum;                       // [T * H] scratch: D = dO . O
+  float* dq_acc;                     // [T * H, d] scratch: fp32 dQ accumulator
+  void *dq, *dk, *dv;                // bf16 outputs
+  int* status;
+  int T, H, G, d, B, topk, NB, num_sms;
+  float scale;
+  unsigned long long wait_ns = 0;
+};
+// D = dO . O and the zeroed dQ accumulator; the key-stationary dK / dV kernel; the
+// query-stationary dQ kernel; dQ converted to bf16.
+cudaError_t launch_bwd_pre(const BwdLaunch& L, cudaStream_t stream);
+cudaError_t launch_bwd_dkdv(const BwdLaunch& L, cudaStream_t stream);
+cudaError_t launch_bwd_dq(const BwdLaunch& L, cudaStream_t stream);
+cudaError_t launch_bwd_finish(const BwdLaunch& L, cudaStream_t stream);
 
 // Whole forward pass on a caller-provided workspace (the body of moba_attn_fwd); the partial
 // outputs of one query chunk are kept under `partial_budget` bytes.

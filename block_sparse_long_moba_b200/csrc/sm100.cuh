@@ -52,14 +52,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // A wait that cannot hang: it gives up after `timeout_ns` (or as soon as another role of the CTA
 // has given up and raised *abort), records `code` in the global error word and returns false.
+// The clock and the abort flag are read every 64 retries (a retry can itself suspend for a
+// while), and on every retry when the limit is below a millisecond (a diagnostic setting), so
+// that a short limit is honoured even by waits that would have succeeded a few retries later.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort_flag, int* err_word,
                                                   int code, uint64_t timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  const bool every = timeout_ns < 1000000ull;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
+    if (every || (it & 63u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > timeout_ns) {
         *abort_flag = 1;

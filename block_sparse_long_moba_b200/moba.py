@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libmoba.so")
 STATUS = {0: "MOBA_OK", -1: "MOBA_ERR_ARG", -2: "MOBA_ERR_UNSUPPORTED", -3: "MOBA_ERR_WORKSPACE",
           -4: "MOBA_ERR_CUDA", -5: "MOBA_ERR_DEVICE_CHECK", -6: "MOBA_ERR_TIMEOUT"}
 KERNEL_CLASSES = ["centroid", "gate", "route_count", "route_scan", "route_scatter", "attention",
-                  "merge", "plan", "densify", "decode"]
+                  "merge", "plan", "densify", "decode", "bwd_dkdv", "bwd_dq", "bwd_aux"]
 
 # every symbol include/moba.h declares
 EXPORTS = ["moba_status_string", "moba_version", "moba_workspace_bytes", "moba_centroids",
@@ -26,7 +26,8 @@ EXPORTS = ["moba_status_string", "moba_version", "moba_workspace_bytes", "moba_c
            "moba_timing_reset", "moba_timing_read", "moba_launch_count",
            "moba_attn_fwd_noalloc", "moba_noalloc_status", "moba_set_wait_limit_ns",
            "moba_centroids_kconv", "moba_attn_fwd_kconv", "moba_decode_workspace_bytes",
-           "moba_decode_fwd"]
+           "moba_decode_fwd", "moba_bwd_workspace_bytes", "moba_attn_bwd",
+           "moba_set_diag_stall"]
 
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -80,10 +81,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moba_decode_fwd.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, P, P, S,
                                     P]
     lib.moba_decode_fwd.restype = I
+    lib.moba_bwd_workspace_bytes.argtypes = [I, P, I, I, I, I, I]
+    lib.moba_bwd_workspace_bytes.restype = S
+    lib.moba_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, P, S, P]
+    lib.moba_attn_bwd.restype = I
     lib.moba_noalloc_status.argtypes = [P]
     lib.moba_noalloc_status.restype = I
     lib.moba_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
     lib.moba_set_wait_limit_ns.restype = ctypes.c_ulonglong
+    lib.moba_set_diag_stall.argtypes = [I]
+    lib.moba_set_diag_stall.restype = I
     _lib = lib
     return lib
 
@@ -392,6 +399,50 @@ def moba_decode_fwd(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
     return o, lse
 
 
+def moba_bwd_workspace_bytes(cu_seqlens_host, hq: int, hkv: int, d: int, block_size: int,
+                             topk: int) -> int:
+    arr, nseq = _host_cu(cu_seqlens_host)
+    return int(load_library().moba_bwd_workspace_bytes(nseq, arr, hq, hkv, d, block_size, topk))
+
+
+def moba_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                  lse: torch.Tensor, d_o: torch.Tensor, block_idx: torch.Tensor,
+                  cu_seqlens: torch.Tensor, cu_seqlens_host, block_size: int, topk: int,
+                  scale: Optional[float] = None, dq: Optional[torch.Tensor] = None,
+                  dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None):
+    """Gradients (dq, dk, dv) of the routed attention with the routing held fixed; o and lse are
+    the forward pass's outputs and block_idx the routing it used."""
+    what = "moba_attn_bwd"
+    arr, nseq = _host_cu(cu_seqlens_host)
+    dev, T, hq, hkv, d = _check_qkv(what, q, k, v, cu_seqlens, nseq)
+    _want(what, "o", o, torch.bfloat16, (T, hq, d), dev)
+    _want(what, "d_o", d_o, torch.bfloat16, (T, hq, d), dev)
+    _want(what, "lse", lse, torch.float32, (hq, T), dev)
+    _want(what, "block_idx", block_idx, torch.int32, (hq, T, topk), dev)
+    if scale is None:
+        scale = d ** -0.5
+    lib = load_library()
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _want(what, "dq", dq, torch.bfloat16, (T, hq, d), dev)
+    _want(what, "dk", dk, torch.bfloat16, (T, hkv, d), dev)
+    _want(what, "dv", dv, torch.bfloat16, (T, hkv, d), dev)
+    if workspace is None:
+        nbytes = int(lib.moba_bwd_workspace_bytes(nseq, arr, hq, hkv, d, block_size, topk))
+        if nbytes == 0 and T > 0:
+            raise MobaError(-1, "moba_bwd_workspace_bytes")
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    _want(what, "workspace", workspace, torch.uint8, None, dev)
+    st = lib.moba_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(d_o),
+                           _ptr(block_idx), _ptr(cu_seqlens), arr, nseq, hq, hkv, d, block_size,
+                           topk, ctypes.c_float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
+                           _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check(st, what)
+    return dq, dk, dv
+
+
 def moba_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                           cu_seqlens: torch.Tensor, cu_seqlens_host, block_size: int, topk: int,
                           scale: Optional[float] = None, o: Optional[torch.Tensor] = None,
@@ -431,6 +482,12 @@ def set_wait_limit_ns(ns: int) -> int:
     """Diagnostics: limit of one pipeline wait in the attention kernel (0 = built-in 2 s);
     returns the previous limit."""
     return int(load_library().moba_set_wait_limit_ns(ctypes.c_ulonglong(int(ns))))
+
+
+def set_diag_stall(on: bool) -> bool:
+    """Diagnostics: make the attention kernel's MMA issuer wait on a barrier nothing arrives on
+    (so that a short wait limit runs out); returns the previous setting."""
+    return bool(load_library().moba_set_diag_stall(1 if on else 0))
 
 
 def timing_enable(on: bool = True):

@@ -185,6 +185,31 @@ int moba_decode_fwd(const void* q, const void* k_cache, const void* v_cache,
                     size_t workspace_bytes, void* stream);
 
 /*
+ * Backward pass of the routed attention [MoBA README, "Introducing MoBA": trainable block sparse
+ * attention]. The routing is held fixed: the top-k gate is piecewise constant in q and the
+ * centroids, so no gradient flows through the selection (as in top-k mixture-of-experts routing).
+ * For every row (t, h) over its attended keys u (the keys of its selected blocks, causal inside
+ * its own block), with p_u = exp(scale q.k_u - lse[h, t]), D = dO[t,h] . o[t,h] and
+ * dS_u = p_u (dO[t,h] . v_u - D):
+ *   dq[t, h] = scale sum_u dS_u k_u,  dk[u, g] = scale sum dS_u q[t, h],  dv[u, g] = sum p_u dO,
+ * the last two summed over every row that attends u and every query head h of kv group g.
+ * q, k, v, o, d_o: bf16 as in moba_attn_fwd (o and lse are that call's outputs; d_o [T, Hq, d]);
+ * block_idx: the routing the forward pass used ([Hq, T, topk], same contract as block_idx_in; a
+ * row that breaks it is reported by moba_device_status as MOBA_ERR_DEVICE_CHECK);
+ * dq [T, Hq, d], dk, dv [T, Hkv, d]: bf16 outputs (fp32 accumulation; dq through an fp32
+ * accumulator in the workspace, dk / dv in tensor memory, each key row written once).
+ * workspace: at least moba_bwd_workspace_bytes(...) bytes, 256-byte aligned (routing lists of all
+ * rows, D and the fp32 dq accumulator). T * Hq * topk < 2^31.
+ */
+size_t moba_bwd_workspace_bytes(int nseq, const int32_t* cu_seqlens_host, int Hq, int Hkv, int d,
+                                int block_size, int topk);
+int moba_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                  const void* d_o, const int32_t* block_idx, const int32_t* cu_seqlens_dev,
+                  const int32_t* cu_seqlens_host, int nseq, int Hq, int Hkv, int d,
+                  int block_size, int topk, float scale, void* dq, void* dk, void* dv,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * moba_attn_fwd for callers that cannot allocate device memory. The paper has no counterpart:
  * this is a deployment variant of the same computation.
  *
@@ -237,6 +262,16 @@ int moba_device_status(const void* workspace, void* stream);
 unsigned long long moba_set_wait_limit_ns(unsigned long long ns);
 
 /*
+ * Diagnostics: with on != 0, later moba_attn_fwd calls make the attention kernel's MMA issuer
+ * first wait on a barrier that nothing arrives on. The wait runs out after the pipeline-wait
+ * limit (set a short one with moba_set_wait_limit_ns), the CTA raises its abort flag, every other
+ * role gives up its own wait, drains its copies in flight and returns, and moba_device_status
+ * reports MOBA_ERR_TIMEOUT: a way to exercise the abort path without a fault. Process-wide;
+ * returns the previous setting. Never set in normal use.
+ */
+int moba_set_diag_stall(int on);
+
+/*
  * Instrumentation (off by default; on from the start when the environment sets MOBA_TIMING=1).
  * When enabled, every kernel launch of the library is bracketed by CUDA events recorded on the
  * launching stream. Every launch is also bracketed by an NVTX range named for its class
@@ -246,8 +281,9 @@ unsigned long long moba_set_wait_limit_ns(unsigned long long ns);
  * recorded events and writes, for each kernel class, the summed device milliseconds and launch
  * count since the last reset; kernel classes, in order: centroid, gate, route_count, route_scan,
  * route_scatter, attention, merge, plan, densify (d = 64: the routed query rows copied into one
- * dense array), decode (moba_decode_fwd's kernels). Returns the number of classes (10), or a
- * negative status.
+ * dense array), decode (moba_decode_fwd's kernels), bwd_dkdv, bwd_dq and bwd_aux (moba_attn_bwd's
+ * key-stationary and query-stationary kernels, and its D / dQ conversion passes). Returns the
+ * number of classes (13), or a negative status.
  */
 int moba_timing_enable(int enable);
 int moba_timing_reset(void);

@@ -115,8 +115,8 @@ def test_timing_classes_match_the_binding(lib):
     from block_sparse_long_moba_b200 import moba
     assert lib.moba_timing_reset() == 0
     n = lib.moba_timing_read(None, None, 0)
-    assert n == len(moba.KERNEL_CLASSES) == 10
-    assert moba.KERNEL_CLASSES[-2:] == ["densify", "decode"]
+    assert n == len(moba.KERNEL_CLASSES) == 13
+    assert moba.KERNEL_CLASSES[-5:] == ["densify", "decode", "bwd_dkdv", "bwd_dq", "bwd_aux"]
 
 
 @pytest.mark.parametrize("value,was_on", [("1", "1"), ("0", "0"), (None, "0")])
