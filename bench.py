@@ -371,7 +371,11 @@ def physical_gpu_index(local: int) -> int:
 # ----------------------------------------------------------------------------------- our arm
 # Workloads timed beside the headline one (one GPU only): the 1M-token shape the metric is also
 # quoted on and the two small-block shapes, each on its own buffers (freed before the next).
-EXTRA_WORKLOADS = (("llama8b_1m", 3), ("routing_64k_b128", 10), ("varlen_512k_b128", 10))
+# The 10M-token record is one rank's share of an 8-way head-parallel split (one kv head and its
+# four query heads of the Llama-3.1-8B shape over the whole sequence): the 8-GPU job runs eight
+# such independent shards.
+EXTRA_WORKLOADS = (("llama8b_1m", 3), ("routing_64k_b128", 10), ("varlen_512k_b128", 10),
+                   ("llama8b_10m_shard8", 2))
 
 
 def measure(w: wl.Workload, steps: int, warmup: int, world: int, rank: int, local: int,

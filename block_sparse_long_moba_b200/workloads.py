@@ -66,6 +66,10 @@ WORKLOADS = {
     "routing_64k_b128": Workload("routing_64k_b128", [0, 65536], 16, 16, 64, 128, 16, "clusters"),
     "varlen_512k_b128": Workload("varlen_512k_b128", [0, 65536, 196608, 294912, 524288],
                                  16, 16, 64, 128, 32, "clusters"),
+    # 10M tokens of the Llama-3.1-8B shape, one rank's share of an 8-way head split (one kv head
+    # and its four query heads; MoBA paper summary, "Key results": attention time at 10M tokens)
+    "llama8b_10m_shard8": Workload("llama8b_10m_shard8", [0, 10485760], 4, 1, 128, 4096, 12,
+                                   "offset"),
     # small cases of the same kernels for profiler captures (a few GB on the device)
     "profile_32k_b4096": Workload("profile_32k_b4096", [0, 32768], 32, 8, 128, 4096, 4, "offset"),
     "profile_32k_b128": Workload("profile_32k_b128", [0, 32768], 16, 16, 64, 128, 16, "clusters"),

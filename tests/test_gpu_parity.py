@@ -172,7 +172,8 @@ def test_empty_input_is_a_noop(moba):
 
 
 # ------------------------------------------------------------------ full-size, sampled rows
-FULL = ["tiny_1k", "routing_64k_b128", "llama8b_128k", "varlen_512k_b128", "llama8b_1m"]
+FULL = ["tiny_1k", "routing_64k_b128", "llama8b_128k", "varlen_512k_b128", "llama8b_1m",
+        "llama8b_10m_shard8"]
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -291,3 +292,35 @@ def test_wait_that_runs_out_reports_timeout_and_the_context_survives(moba, d):
                                    tokens)
     pu.check_outputs(o.cpu().float().numpy(), lse.cpu().numpy(), o_ref, lse_ref)
 
+
+
+# ------------------------------------------------------------------------- head-parallel split
+def test_head_shards_reproduce_the_whole_problem(moba):
+    """Running moba_attn_fwd on each rank's share of the heads (the head-parallel split, ranks
+    emulated one after another on this GPU; no rank waits on another) and concatenating the heads
+    gives the whole problem's result: the same routing and O / LSE within the parity tolerance of
+    the single run."""
+    from block_sparse_long_moba_b200 import shard
+
+    cu = [0, 5000, 5000, 12000]
+    hq, hkv, d, B, topk = 8, 4, 128, 512, 4
+    w, q, k, v, cu_t = _inputs(cu, hq, hkv, d, B, topk, "clusters")
+    idx = torch.empty((hq, cu[-1], topk), dtype=torch.int32, device="cuda")
+    o, lse = moba.moba_attn_fwd(q, k, v, cu_t, cu, B, topk, block_idx_out=idx)
+    for world in (2, 4):
+        parts_o, parts_l, parts_i = [], [], []
+        for rank in range(world):
+            ql, kl, vl = shard.take_heads(q, k, v, world, rank)
+            il = torch.empty((ql.shape[1], cu[-1], topk), dtype=torch.int32, device="cuda")
+            ol, ll = shard.moba_attn_fwd_heads(ql, kl, vl, cu_t, cu, B, topk, block_idx_out=il)
+            parts_o.append(ol)
+            parts_l.append(ll)
+            parts_i.append(il)
+        torch.cuda.synchronize()
+        o2, l2, i2 = torch.cat(parts_o, 1), torch.cat(parts_l, 0), torch.cat(parts_i, 0)
+        mism = (i2 != idx).any(dim=2)
+        assert mism.float().mean().item() <= pu.TIE_ROWS_MAX, mism.sum().item()
+        ok = ~mism.T[:, :, None].expand_as(o)
+        err = (o2.float() - o.float()).abs()
+        assert (err[ok] <= pu.O_ATOL + pu.O_RTOL * o.float().abs()[ok]).all()
+        assert ((l2 - lse).abs()[~mism] <= pu.LSE_ATOL).all()
