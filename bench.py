@@ -826,11 +826,23 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-extra", action="store_true",
                     help="time only --workload (skip the 1M and small-block sub-records)")
-    ap.add_argument("--only", choices=["gate"], default=None,
-                    help="time centroids + gate alone (1 GPU; for profiling)")
+    ap.add_argument("--only", choices=["gate", "backward", "decode"], default=None,
+                    help="time one part alone on --workload (1 GPU; for profiling): centroids + "
+                         "gate, the backward pass, or decode")
     args = ap.parse_args()
     if args.only == "gate":
         run_gate_only(args)
+    elif args.only in ("backward", "decode"):
+        from block_sparse_long_moba_b200 import build, moba
+        build.build()
+        moba.load_library()
+        torch.cuda.set_device(0)
+        peaks = read_peaks()
+        if args.only == "backward":
+            rec = measure_backward(wl.WORKLOADS[args.workload], args.steps, args.warmup, peaks)
+        else:
+            rec = measure_decode(args.steps, args.warmup, peaks)
+        print(json.dumps(rec), flush=True)
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -581,17 +581,63 @@ int moba_decode_fwd(const void* q, const void* k_cache, const void* v_cache,
 
 namespace {
 
-struct BwdLayout {
-  size_t status, blk_off, blk_seq, blk_start, blk_len, counts, cursor, tiles, entries, dsum, dq_acc,
-      total;
+constexpr size_t kBwdDenseBudgetBytes = 16ull << 30;  // routed rows of one chunk, densified
+
+// Host-side plan of the backward pass: query chunks of whole blocks whose routed entries, with
+// their densified query / dO rows and per-row columns, fit the budget.
+struct BwdPlan {
+  Plan P;
+  std::vector<Chunk> chunks;
+  size_t max_entries = 0;   // largest chunk
+  size_t last_entries = 0;  // the chunk being filled
 };
 
-BwdLayout bwd_layout(const Plan& P, int nseq, int Hq, int Hkv, int d, int topk) {
+int bwd_plan(int nseq, const int32_t* cu, int Hq, int Hkv, int d, int B, int topk, BwdPlan* BP) {
+  int st = check_cu(nseq, cu);
+  if (st != MOBA_OK) return st;
+  if ((st = check_shape(Hq, Hkv, d, B, topk)) != MOBA_OK) return st;
+  if ((st = make_plan(nseq, cu, Hq, Hkv, d, B, topk, &BP->P, ~static_cast<size_t>(0) >> 1)) !=
+      MOBA_OK)
+    return st;
+  const size_t per_entry = 4 + static_cast<size_t>(d) * 4 + 12;
+  const size_t max_ent = std::max<size_t>(kBwdDenseBudgetBytes / per_entry, 1);
+  BP->chunks.clear();
+  BP->max_entries = 0;
+  int b = 0, t = 0;
+  for (int s = 0; s < nseq; ++s) {
+    const int L = cu[s + 1] - cu[s];
+    for (int i = 0; i < blocks_of(L, B); ++i, ++b) {
+      const int n = std::min(B, L - i * B);
+      const size_t ent = static_cast<size_t>(n) * Hq * (std::min(topk, i + 1) - 1);
+      if (BP->chunks.empty() ||
+          (BP->chunks.back().nblk > 0 && BP->last_entries + ent > max_ent)) {
+        BP->chunks.push_back(Chunk{b, 0, t, 0});
+        BP->last_entries = 0;
+      }
+      Chunk& c = BP->chunks.back();
+      c.nblk += 1;
+      c.ntok += n;
+      BP->last_entries += ent;
+      BP->max_entries = std::max(BP->max_entries, BP->last_entries);
+      if (static_cast<long long>(c.ntok) * Hq * topk >= (1LL << 31)) return MOBA_ERR_UNSUPPORTED;
+      t += n;
+    }
+  }
+  return MOBA_OK;
+}
+
+struct BwdLayout {
+  size_t status, blk_off, blk_seq, blk_start, blk_len, counts, cursor, tiles, entries, qd, dd,
+      col_lse, col_d, col_t, dsum, dq_acc, dk_acc, dv_acc, total;
+};
+
+BwdLayout bwd_layout(const BwdPlan& BP, int nseq, int Hq, int Hkv, int d) {
+  const Plan& P = BP.P;
   BwdLayout L;
   size_t o = 0;
   auto take = [&](size_t bytes) { const size_t at = o; o = up256(o + bytes); return at; };
   const size_t rows = static_cast<size_t>(P.T) * Hq;
-  const size_t ent = rows * (topk - 1);
+  const size_t ent = std::max<size_t>(BP.max_entries, 1);
   L.status = take(256);
   L.blk_off = take(static_cast<size_t>(nseq + 1) * 4);
   L.blk_seq = take(static_cast<size_t>(P.NB) * 4);
@@ -600,23 +646,18 @@ BwdLayout bwd_layout(const Plan& P, int nseq, int Hq, int Hkv, int d, int topk) 
   L.counts = take(static_cast<size_t>(Hkv) * P.NB * 4);
   L.cursor = take(static_cast<size_t>(Hkv) * P.NB * 4);
   L.tiles = take((ent / kItemRows + static_cast<size_t>(Hkv) * P.NB + 1) * 16);
-  L.entries = take(std::max<size_t>(ent, 1) * 4);
+  L.entries = take(ent * 4);
+  L.qd = take(ent * d * 2);
+  L.dd = take(ent * d * 2);
+  L.col_lse = take(ent * 4);
+  L.col_d = take(ent * 4);
+  L.col_t = take(ent * 4);
   L.dsum = take(rows * 4);
   L.dq_acc = take(rows * d * 4);
+  L.dk_acc = take(static_cast<size_t>(P.T) * Hkv * d * 4);
+  L.dv_acc = take(static_cast<size_t>(P.T) * Hkv * d * 4);
   L.total = o;
   return L;
-}
-
-int bwd_check(int nseq, const int32_t* cu_host, int Hq, int Hkv, int d, int B, int topk, Plan* P) {
-  int st = check_cu(nseq, cu_host);
-  if (st != MOBA_OK) return st;
-  if ((st = check_shape(Hq, Hkv, d, B, topk)) != MOBA_OK) return st;
-  // one query chunk over the whole problem: the routing lists of every row at once
-  if ((st = make_plan(nseq, cu_host, Hq, Hkv, d, B, topk, P, ~static_cast<size_t>(0) >> 1)) !=
-      MOBA_OK)
-    return st;
-  if (static_cast<long long>(P->T) * Hq * topk >= (1LL << 31)) return MOBA_ERR_UNSUPPORTED;
-  return MOBA_OK;
 }
 
 }  // namespace
@@ -625,9 +666,9 @@ extern "C" {
 
 size_t moba_bwd_workspace_bytes(int nseq, const int32_t* cu_seqlens_host, int Hq, int Hkv, int d,
                                 int block_size, int topk) {
-  Plan P;
-  if (bwd_check(nseq, cu_seqlens_host, Hq, Hkv, d, block_size, topk, &P) != MOBA_OK) return 0;
-  return bwd_layout(P, nseq, Hq, Hkv, d, topk).total;
+  BwdPlan BP;
+  if (bwd_plan(nseq, cu_seqlens_host, Hq, Hkv, d, block_size, topk, &BP) != MOBA_OK) return 0;
+  return bwd_layout(BP, nseq, Hq, Hkv, d).total;
 }
 
 int moba_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -635,9 +676,10 @@ int moba_attn_bwd(const void* q, const void* k, const void* v, const void* o, co
                   const int32_t* cu_host, int nseq, int Hq, int Hkv, int d, int block_size,
                   int topk, float scale, void* dq, void* dk, void* dv, void* workspace,
                   size_t workspace_bytes, void* stream) {
-  Plan P;
-  int st = bwd_check(nseq, cu_host, Hq, Hkv, d, block_size, topk, &P);
+  BwdPlan BP;
+  int st = bwd_plan(nseq, cu_host, Hq, Hkv, d, block_size, topk, &BP);
   if (st != MOBA_OK) return st;
+  const Plan& P = BP.P;
   if (!(scale > 0.f) || scale > 1e30f) return MOBA_ERR_ARG;
   if (P.T == 0) return MOBA_OK;
   const void* ptrs[] = {q, k, v, o, lse, d_o, block_idx, dq, dk, dv};
@@ -645,7 +687,7 @@ int moba_attn_bwd(const void* q, const void* k, const void* v, const void* o, co
     if (!p || !aligned16(p)) return MOBA_ERR_ARG;
   if (!cu_dev || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return MOBA_ERR_ARG;
-  const BwdLayout L = bwd_layout(P, nseq, Hq, Hkv, d, topk);
+  const BwdLayout L = bwd_layout(BP, nseq, Hq, Hkv, d);
   if (workspace_bytes < L.total) return MOBA_ERR_WORKSPACE;
   int sms = 0;
   if ((st = device_check(&sms)) != MOBA_OK) return st;
@@ -662,27 +704,40 @@ int moba_attn_bwd(const void* q, const void* k, const void* v, const void* o, co
   int4* tiles = at<int4>(workspace, L.tiles);
   int* entries = at<int>(workspace, L.entries);
   const int NBK = Hkv * P.NB;
-  MOBA_LAUNCH(kPlan, s, launch_plan(cu_dev, nseq, block_size, P.NB, tb, counts, NBK, status, s));
-  MOBA_LAUNCH(kRouteCount, s,
-              launch_route_count(block_idx, tb, P.T, Hq, Hkv, topk, P.NB, 0, P.NB, 0, P.max_nb,
-                                 counts, status, s));
-  MOBA_LAUNCH(kRouteScan, s, launch_route_scan(counts, NBK, cursor, tiles, n_tiles, s));
-  MOBA_LAUNCH(kRouteScatter, s,
-              launch_route_scatter(block_idx, tb, P.T, Hq, Hkv, topk, P.NB, 0, P.NB, 0, P.max_nb,
-                                   cursor, entries, s));
   BwdLaunch B;
   B.q = q; B.k = k; B.v = v; B.o = o; B.dout = d_o; B.lse = lse;
   B.entries = entries; B.bucket_end = cursor; B.tiles = tiles; B.n_routed = n_tiles;
   B.tb = tb;
   B.dsum = at<float>(workspace, L.dsum);
   B.dq_acc = at<float>(workspace, L.dq_acc);
+  B.dk_acc = at<float>(workspace, L.dk_acc);
+  B.dv_acc = at<float>(workspace, L.dv_acc);
+  B.qd = at<void>(workspace, L.qd);
+  B.dd = at<void>(workspace, L.dd);
+  B.col_lse = at<float>(workspace, L.col_lse);
+  B.col_d = at<float>(workspace, L.col_d);
+  B.col_t = at<int>(workspace, L.col_t);
+  B.dense_rows = static_cast<long long>(std::max<size_t>(BP.max_entries, 1));
   B.dq = dq; B.dk = dk; B.dv = dv; B.status = status;
   B.T = P.T; B.H = Hq; B.G = Hkv; B.d = d; B.B = block_size; B.topk = topk; B.NB = P.NB;
   B.num_sms = sms; B.scale = scale;
+  B.T0 = 0; B.b0 = 0; B.nblk = P.NB;
   B.wait_ns = g_wait_limit_ns.load();
+  MOBA_LAUNCH(kPlan, s, launch_plan(cu_dev, nseq, block_size, P.NB, tb, counts, NBK, status, s));
   MOBA_LAUNCH(kBwdAux, s, launch_bwd_pre(B, s));
-  MOBA_LAUNCH(kBwdDkdv, s, launch_bwd_dkdv(B, s));
-  MOBA_LAUNCH(kBwdDq, s, launch_bwd_dq(B, s));
+  for (const Chunk& c : BP.chunks) {
+    B.T0 = c.T0; B.b0 = c.b0; B.nblk = c.nblk;
+    MOBA_LAUNCH(kRouteCount, s,
+                launch_route_count(block_idx, tb, P.T, Hq, Hkv, topk, P.NB, c.b0, c.nblk, c.T0,
+                                   P.max_nb, counts, status, s));
+    MOBA_LAUNCH(kRouteScan, s, launch_route_scan(counts, NBK, cursor, tiles, n_tiles, s));
+    MOBA_LAUNCH(kRouteScatter, s,
+                launch_route_scatter(block_idx, tb, P.T, Hq, Hkv, topk, P.NB, c.b0, c.nblk, c.T0,
+                                     P.max_nb, cursor, entries, s));
+    MOBA_LAUNCH(kBwdAux, s, launch_bwd_densify(B, s));
+    MOBA_LAUNCH(kBwdDkdv, s, launch_bwd_dkdv(B, s));
+    MOBA_LAUNCH(kBwdDq, s, launch_bwd_dq(B, s));
+  }
   MOBA_LAUNCH(kBwdAux, s, launch_bwd_finish(B, s));
   return MOBA_OK;
 }

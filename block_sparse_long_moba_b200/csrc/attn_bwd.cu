@@ -6,12 +6,19 @@
 //   dV[u] += p_u dO,   dK[u] += scale dS_u q,   dQ += scale sum_u dS_u k_u,
 // and a kv head's dK / dV collect the terms of every query head of its group.
 //
+// The query range is processed in chunks of whole blocks (as in the forward pass), so that the
+// routing lists and the densified rows of one chunk fit a fixed memory budget.
 //   bwd_pre_kernel   D = dO . O per row (fp32), and the fp32 dQ accumulator zeroed.
+//   bwd_densify      per chunk: the query and dO rows of every routed entry copied in list order
+//                    into dense arrays, with the row's log2-domain LSE, D and position, so that a
+//                    routed query tile is one 128-row TMA tile load [FlashMoBA story, Gather-and-
+//                    Densify] — every key sub-tile of the block reads the same tiles again.
 //   bwd_dkdv_kernel  key-stationary: one work item per (kv head g, block b, 128-key sub-tile j)
-//                    walks every 128-row query tile that attends those keys — the rows routed to b
-//                    (the routing inversion's list of (g, b), gathered from scattered rows) and the
-//                    rows of block b itself at or after the sub-tile (causal) — and keeps dK, dV of
-//                    its 128 keys in tensor memory; each key row has one owner, so no atomics:
+//                    walks every 128-row query tile of the chunk that attends those keys — the rows
+//                    routed to b (dense tiles) and the rows of block b itself at or after the
+//                    sub-tile (causal; 128 consecutive tokens of one head, a strided TMA tile) —
+//                    and keeps dK, dV of its 128 keys in tensor memory, then adds them to the fp32
+//                    dK, dV rows it owns (one owner per row in a launch: no atomics):
 //                      S^T  = K_j Q^T      (M = 128 keys, N = 128 rows, K = d)
 //                      dP^T = V_j dO^T
 //                      P^T  = exp2(S^T scale log2e - LSE2), dS^T = P^T (dP^T - D), written back
@@ -23,7 +30,7 @@
 //                      dQ += dS K_j
 //                    and adds scale * dQ once per item into the fp32 accumulator (red.global.add;
 //                    a row collects one addition per selected block).
-//   bwd_dq_finish    dQ = bf16(accumulator).
+//   bwd_finish       dQ, dK, dV = bf16(accumulators).
 // Warp roles (256 threads): warp 0 = TMA producer (tiles and, for the query tiles, the per-row
 // LSE / D / position columns), warp 1 = TMEM owner and MMA issuer, warps 4-7 = one thread per
 // tensor-memory lane (the elementwise softmax-gradient step and the epilogues). Every wait is
@@ -43,16 +50,20 @@ constexpr int kOneCtaPerSmBytes = 120 * 1024;  // more than half of an SM's shar
 struct BwdArgs {
   const float* lse;         // [H, T] natural log
   const float* dsum;        // [T * H] D = dO . O
-  const int* entries;       // routed entries ((t * H + h) * topk + slot), grouped by (g, b)
-  const int* bucket_end;    // [G * NB] end offset of every (g, b) list
+  const int* entries;       // chunk's routed entries (((t - T0) * H + h) * topk + slot) by (g, b)
+  const int* bucket_end;    // [G * NB] end offset of every (g, b) list of the chunk
   const int4* tiles;        // routed 256-row items {bucket, first entry, rows}
   const int* n_routed;      // device count of routed items
+  const float* col_lse;     // densified entries: log2-domain LSE, D and position of each row
+  const float* col_d;
+  const int* col_t;
   BlockTables tb;
-  __nv_bfloat16* dk;        // [T, G, D]
-  __nv_bfloat16* dv;
   float* dq_acc;            // [T * H, D]
+  float* dk_acc;            // [T, G, D]
+  float* dv_acc;
   int* status;
   int T, H, G, r, topk, NB, SPB;
+  int T0, b0, nblk;         // the chunk: first token, first query block, query blocks
   float scale_log2, scale;
   unsigned long long wait_ns;
 };
@@ -96,13 +107,48 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
   for (int e = 0; e < PER; ++e) dq_acc[row * D + lane * PER + e] = 0.f;
 }
 
-__global__ void __launch_bounds__(256) bwd_dq_finish_kernel(const float4* __restrict__ acc,
-                                                            long long n4,
-                                                            uint2* __restrict__ dq) {
+__global__ void __launch_bounds__(256) bwd_zero_kernel(float4* __restrict__ p, long long n4) {
+  for (long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; x < n4;
+       x += static_cast<long long>(gridDim.x) * blockDim.x)
+    p[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+__global__ void __launch_bounds__(256) bwd_finish_kernel(const float4* __restrict__ acc,
+                                                         long long n4, uint2* __restrict__ out) {
   for (long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; x < n4;
        x += static_cast<long long>(gridDim.x) * blockDim.x) {
     const float4 a = acc[x];
-    dq[x] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+    out[x] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+  }
+}
+
+// Densify one chunk's routed entries: dense row p = query row and dO row of entry p, plus the
+// row's log2-domain LSE, D and position. Consecutive entries go to consecutive rows (coalesced
+// 16-byte stores, D / 8 lanes per row); the source rows are read at random.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_densify_kernel(
+    const int* __restrict__ entries, const int* __restrict__ n_entries,
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ dout,
+    const float* __restrict__ lse, const float* __restrict__ dsum, int T, int H, int topk, int T0,
+    __nv_bfloat16* __restrict__ qd, __nv_bfloat16* __restrict__ dd, float* __restrict__ col_lse,
+    float* __restrict__ col_d, int* __restrict__ col_t) {
+  constexpr int LPR = D / 8;  // lanes per row
+  const int n = *n_entries;
+  const int sub = threadIdx.x % LPR;
+  const long long stride = static_cast<long long>(gridDim.x) * (blockDim.x / LPR);
+  for (long long p = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / LPR; p < n;
+       p += stride) {
+    const long long row = static_cast<long long>(T0) * H + __ldg(entries + p) / topk;
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(q + row * D) + sub);
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + sub);
+    __stcs(reinterpret_cast<uint4*>(qd + p * D) + sub, a);
+    __stcs(reinterpret_cast<uint4*>(dd + p * D) + sub, b);
+    if (sub == 0) {
+      const int t = static_cast<int>(row / H), h = static_cast<int>(row % H);
+      col_lse[p] = __ldg(lse + static_cast<size_t>(h) * T + t) * 1.4426950408889634f;
+      col_d[p] = __ldg(dsum + row);
+      col_t[p] = t;
+    }
   }
 }
 
@@ -121,20 +167,21 @@ struct KvItem {
 __device__ __forceinline__ KvItem kv_item(const BwdArgs& a, int w) {
   KvItem it;
   it.j = w % a.SPB;
-  const int bg = w / a.SPB;
-  it.g = bg % a.G;
-  it.b = bg / a.G;
+  const int x = w / a.SPB;  // bucket g * NB + b: a bucket's sub-tiles are consecutive items
+  it.g = x / a.NB;
+  it.b = x % a.NB;
   const int bstart = a.tb.blk_start[it.b], blen = a.tb.blk_len[it.b];
-  it.valid = it.j * 128 < blen;
   it.key0 = bstart + it.j * 128;
   it.klen = min(128, blen - it.j * 128);
   it.bend = bstart + blen;
-  const int x = it.g * a.NB + it.b;
   it.rstart = x > 0 ? a.bucket_end[x - 1] : 0;
   it.rcount = a.bucket_end[x] - it.rstart;
   it.nrt = (it.rcount + 127) / 128;
-  it.ndt_head = (it.bend - it.key0 + 127) / 128;
+  // the block's own rows belong to the chunk that holds the block
+  const bool own = it.b >= a.b0 && it.b < a.b0 + a.nblk;
+  it.ndt_head = own ? (it.bend - it.key0 + 127) / 128 : 0;
   it.ntile = it.nrt + a.r * it.ndt_head;
+  it.valid = it.j * 128 < blen && it.ntile > 0;
   return it;
 }
 
@@ -145,8 +192,8 @@ struct KvCfg {
   static constexpr int OFF_V = TILE;
   static constexpr int OFF_Q = 2 * TILE;             // stage s: Q at OFF_Q + s * 2 TILE
   static constexpr int OFF_DO = 3 * TILE;            //          dO at OFF_DO + s * 2 TILE
-  static constexpr int OFF_COL = 6 * TILE;           // [2 stages][3][128] lse2, D, position
-  static constexpr int OFF_BARS = OFF_COL + 2 * 3 * 128 * 4;
+  static constexpr int OFF_COL = 6 * TILE;           // [2 stages][128] {lse2, D} per column
+  static constexpr int OFF_BARS = OFF_COL + 2 * 128 * 8;
   static constexpr int SMEM = OFF_BARS + 256;
 };
 
@@ -163,12 +210,14 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v,
-                    const __grid_constant__ CUtensorMap map_q,
-                    const __grid_constant__ CUtensorMap map_do, const BwdArgs a, int n_items) {
+                    const __grid_constant__ CUtensorMap map_q3,
+                    const __grid_constant__ CUtensorMap map_do3,
+                    const __grid_constant__ CUtensorMap map_qd,
+                    const __grid_constant__ CUtensorMap map_dd, const BwdArgs a, int n_items) {
   using C = KvCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   KvBars* bars = reinterpret_cast<KvBars*>(smem + C::OFF_BARS);
-  float* col = reinterpret_cast<float*>(smem + C::OFF_COL);  // [stage][lse2 | D | t][128]
+  float2* col = reinterpret_cast<float2*>(smem + C::OFF_COL);  // [stage][128] {lse2, D}
   volatile int* abort_flag = &bars->abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (smem_u32(smem) & 1023u) {
@@ -197,8 +246,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&map_k);
     prefetch_tensormap(&map_v);
-    prefetch_tensormap(&map_q);
-    prefetch_tensormap(&map_do);
+    prefetch_tensormap(&map_q3);
+    prefetch_tensormap(&map_do3);
+    prefetch_tensormap(&map_qd);
+    prefetch_tensormap(&map_dd);
   }
   tc_fence_before();
   __syncthreads();
@@ -234,56 +285,54 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int st = gt & 1;
         ok = wait_all(&bars->qd_empty[st], ((gt >> 1) & 1) ^ 1);
         if (!ok) break;
-        // columns 4 lane .. 4 lane + 3 of the tile: query row (t * H + h), log2-domain LSE, D,
-        // position; padding columns repeat a valid row and get LSE2 = +inf (p = 0)
-        int rows4[4];
-        float* cl = col + st * 3 * 128;
-        int first_row = 0;
-        for (int e = 0; e < 4; ++e) {
-          const int c = 4 * lane + e;
-          int row = -1, t = -1;
-          if (n < it.nrt) {
-            const int m = n * 128 + c;
-            if (m < it.rcount) {
-              row = __ldg(a.entries + it.rstart + m) / a.topk;
-              t = row / a.H;
-            }
-            if (e == 0 && lane == 0) first_row = __ldg(a.entries + it.rstart + n * 128) / a.topk;
-          } else {
-            const int dn = n - it.nrt;
-            const int h = it.g * a.r + dn / it.ndt_head;
-            const int tt = it.key0 + (dn % it.ndt_head) * 128 + c;
-            if (tt < it.bend) {
-              t = tt;
-              row = t * a.H + h;
-            }
-            if (e == 0 && lane == 0) first_row = (it.key0 + (dn % it.ndt_head) * 128) * a.H + h;
-          }
-          rows4[e] = row;
-          if (row >= 0) {
-            cl[c] = __ldg(a.lse + static_cast<size_t>(row % a.H) * a.T + t) * 1.4426950408889634f;
-            cl[128 + c] = __ldg(a.dsum + row);
-            reinterpret_cast<int*>(cl)[256 + c] = t;
-          } else {
-            cl[c] = INFINITY;
-            cl[128 + c] = 0.f;
-            reinterpret_cast<int*>(cl)[256 + c] = -1;
-          }
-        }
-        first_row = __shfl_sync(0xffffffffu, first_row, 0);
+        // columns 4 lane .. 4 lane + 3 of the tile: {log2-domain LSE, D} of the row (padding
+        // columns: LSE2 = +inf, so that p = 0); the rows themselves arrive as one 128-row TMA
+        // tile (dense routed rows, or 128 consecutive tokens of one head)
+        float2* cl = col + st * 128;
+        uint8_t* dq_ = smem + C::OFF_Q + st * 2 * C::TILE;
+        uint8_t* dd_ = smem + C::OFF_DO + st * 2 * C::TILE;
+        if (n < it.nrt) {
+          const int p0 = it.rstart + n * 128;
+          const int rows = min(128, it.rcount - n * 128);
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (rows4[e] < 0) rows4[e] = first_row;
-        if (lane == 0) mbar_arrive_expect_tx(&bars->qd_full[st], 2 * C::TILE);
-        __syncwarp();
-        uint8_t* dq_ = smem + C::OFF_Q + st * 2 * C::TILE + lane * 512;
-        uint8_t* dd_ = smem + C::OFF_DO + st * 2 * C::TILE + lane * 512;
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * lane + e;
+            const bool on = c < rows;
+            cl[c] = make_float2(on ? __ldg(a.col_lse + p0 + c) : INFINITY,
+                                on ? __ldg(a.col_d + p0 + c) : 0.f);
+          }
+          if (lane == 0) mbar_arrive_expect_tx(&bars->qd_full[st], 2 * C::TILE);
+          __syncwarp();
+          if (lane == 0) {
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_gather4(dq_ + c * 16384, &map_q, &bars->qd_full[st], c * 64, rows4[0], rows4[1],
-                      rows4[2], rows4[3]);
-          tma_gather4(dd_ + c * 16384, &map_do, &bars->qd_full[st], c * 64, rows4[0], rows4[1],
-                      rows4[2], rows4[3]);
+            for (int c = 0; c < D / 64; ++c) {
+              tma_load_2d(dq_ + c * 16384, &map_qd, &bars->qd_full[st], c * 64, p0);
+              tma_load_2d(dd_ + c * 16384, &map_dd, &bars->qd_full[st], c * 64, p0);
+            }
+          }
+        } else {
+          const int dn = n - it.nrt;
+          const int h = it.g * a.r + dn / it.ndt_head;
+          const int t0 = it.key0 + (dn % it.ndt_head) * 128;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * lane + e;
+            const int t = t0 + c;
+            const bool on = t < it.bend;
+            cl[c] = make_float2(
+                on ? __ldg(a.lse + static_cast<size_t>(h) * a.T + t) * 1.4426950408889634f
+                   : INFINITY,
+                on ? __ldg(a.dsum + static_cast<size_t>(t) * a.H + h) : 0.f);
+          }
+          if (lane == 0) mbar_arrive_expect_tx(&bars->qd_full[st], 2 * C::TILE);
+          __syncwarp();
+          if (lane == 0) {
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+              tma_load_3d(dq_ + c * 16384, &map_q3, &bars->qd_full[st], c * 64, h, t0);
+              tma_load_3d(dd_ + c * 16384, &map_do3, &bars->qd_full[st], c * 64, h, t0);
+            }
+          }
         }
         mbar_arrive(&bars->qd_full[st]);  // this lane's columns are written
       }
@@ -383,37 +432,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = wait_all(&bars->s_full, gt & 1);
         if (!ok) break;
         tc_fence_after();
-        const float* cl = col + st * 3 * 128;
-        const int* ct = reinterpret_cast<const int*>(cl) + 256;
-#pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-          uint32_t sr[32], dr[32];
-          tmem_ld32(tmem + lane_off + TM_S + c0, sr);
-          tmem_ld32(tmem + lane_off + TM_DP + c0, dr);
-          tmem_wait_ld();
+        const float4* cl4 = reinterpret_cast<const float4*>(col + st * 128);  // 2 columns each
+        // columns c < cmin are queries before this key (the causal cut of the block's own rows:
+        // u <= t0 + c); routed rows all follow the block
+        int cmin = 0;
+        if (n >= it.nrt) cmin = u - (it.key0 + ((n - it.nrt) % it.ndt_head) * 128);
+        if (!kvalid) cmin = 128;
+        // 32-column chunks; the next chunk's tensor-memory loads are in flight while this one is
+        // computed. Packed P / dS of chunk ch go to columns 16 ch .. 16 ch + 15, already read.
+        uint32_t sr[2][32], dr[2][32];
+        tmem_ld32(tmem + lane_off + TM_S, sr[0]);
+        tmem_ld32(tmem + lane_off + TM_DP, dr[0]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const int cur = ch & 1;
+          if (ch < 3) {
+            tmem_ld32(tmem + lane_off + TM_S + 32 * (ch + 1), sr[cur ^ 1]);
+            tmem_ld32(tmem + lane_off + TM_DP + 32 * (ch + 1), dr[cur ^ 1]);
+          }
 #pragma unroll
           for (int x = 0; x < 32; ++x) {
-            reg_fence(sr[x]);
-            reg_fence(dr[x]);
+            reg_fence(sr[cur][x]);
+            reg_fence(dr[cur][x]);
           }
           uint32_t pp[16], dd[16];
 #pragma unroll
           for (int x = 0; x < 32; x += 2) {
-            float p[2], ds[2];
-#pragma unroll
-            for (int y = 0; y < 2; ++y) {
-              const int c = c0 + x + y;
-              const bool on = kvalid && u <= ct[c];
-              p[y] = on ? ex2_approx(fmaf(__uint_as_float(sr[x + y]), sl2, -cl[c])) : 0.f;
-              ds[y] = p[y] * (__uint_as_float(dr[x + y]) - cl[128 + c]);
-            }
-            pp[x >> 1] = pack_bf16x2(p[0], p[1]);
-            dd[x >> 1] = pack_bf16x2(ds[0], ds[1]);
+            const int c = 32 * ch + x;
+            const float4 cc = cl4[c >> 1];  // {lse2, D} of columns c and c + 1
+            const float p0 = c >= cmin ? ex2_approx(fmaf(__uint_as_float(sr[cur][x]), sl2, -cc.x))
+                                       : 0.f;
+            const float p1 = c + 1 >= cmin
+                                 ? ex2_approx(fmaf(__uint_as_float(sr[cur][x + 1]), sl2, -cc.z))
+                                 : 0.f;
+            pp[x >> 1] = pack_bf16x2(p0, p1);
+            dd[x >> 1] = pack_bf16x2(p0 * (__uint_as_float(dr[cur][x]) - cc.y),
+                                     p1 * (__uint_as_float(dr[cur][x + 1]) - cc.w));
           }
-          // packed in place: columns c0/2 .. c0/2 + 15 of S and dP were read by this or an
-          // earlier chunk
-          tmem_st16(tmem + lane_off + TM_S + c0 / 2, pp);
-          tmem_st16(tmem + lane_off + TM_DP + c0 / 2, dd);
+          tmem_st16(tmem + lane_off + TM_S + 16 * ch, pp);
+          tmem_st16(tmem + lane_off + TM_DP + 16 * ch, dd);
+          if (ch < 3) tmem_wait_ld();
         }
         tmem_wait_st();
         tc_fence_before();
@@ -424,8 +483,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = wait_all(&bars->acc_full, li & 1);
       if (!ok) break;
       tc_fence_after();
-      __nv_bfloat16* dkr = a.dk + (static_cast<size_t>(u) * a.G + it.g) * D;
-      __nv_bfloat16* dvr = a.dv + (static_cast<size_t>(u) * a.G + it.g) * D;
+      float* dka = a.dk_acc + (static_cast<size_t>(u) * a.G + it.g) * D;
+      float* dva = a.dv_acc + (static_cast<size_t>(u) * a.G + it.g) * D;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t kr[32], vr[32];
@@ -438,19 +497,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           reg_fence(vr[x]);
         }
         if (kvalid) {
+          // this item owns rows (u, g): earlier chunks' sums are read back and extended
 #pragma unroll
-          for (int x = 0; x < 32; x += 8) {
-            uint4 kk, vv;
-            kk.x = pack_bf16x2(__uint_as_float(kr[x]) * a.scale, __uint_as_float(kr[x + 1]) * a.scale);
-            kk.y = pack_bf16x2(__uint_as_float(kr[x + 2]) * a.scale, __uint_as_float(kr[x + 3]) * a.scale);
-            kk.z = pack_bf16x2(__uint_as_float(kr[x + 4]) * a.scale, __uint_as_float(kr[x + 5]) * a.scale);
-            kk.w = pack_bf16x2(__uint_as_float(kr[x + 6]) * a.scale, __uint_as_float(kr[x + 7]) * a.scale);
-            vv.x = pack_bf16x2(__uint_as_float(vr[x]), __uint_as_float(vr[x + 1]));
-            vv.y = pack_bf16x2(__uint_as_float(vr[x + 2]), __uint_as_float(vr[x + 3]));
-            vv.z = pack_bf16x2(__uint_as_float(vr[x + 4]), __uint_as_float(vr[x + 5]));
-            vv.w = pack_bf16x2(__uint_as_float(vr[x + 6]), __uint_as_float(vr[x + 7]));
-            *reinterpret_cast<uint4*>(dkr + c0 + x) = kk;
-            *reinterpret_cast<uint4*>(dvr + c0 + x) = vv;
+          for (int x = 0; x < 32; x += 4) {
+            float4 kk = *reinterpret_cast<const float4*>(dka + c0 + x);
+            float4 vv = *reinterpret_cast<const float4*>(dva + c0 + x);
+            kk.x = fmaf(__uint_as_float(kr[x]), a.scale, kk.x);
+            kk.y = fmaf(__uint_as_float(kr[x + 1]), a.scale, kk.y);
+            kk.z = fmaf(__uint_as_float(kr[x + 2]), a.scale, kk.z);
+            kk.w = fmaf(__uint_as_float(kr[x + 3]), a.scale, kk.w);
+            vv.x += __uint_as_float(vr[x]);
+            vv.y += __uint_as_float(vr[x + 1]);
+            vv.z += __uint_as_float(vr[x + 2]);
+            vv.w += __uint_as_float(vr[x + 3]);
+            *reinterpret_cast<float4*>(dka + c0 + x) = kk;
+            *reinterpret_cast<float4*>(dva + c0 + x) = vv;
           }
         }
       }
@@ -496,8 +557,8 @@ __device__ __forceinline__ QItem q_item(const BwdArgs& a, int w, int n_routed) {
   const int wd = w - 2 * n_routed;
   it.h = wd % a.H;
   const int rest = wd / a.H;
-  const int bl = rest % a.NB;
-  const int p = a.SPB - 1 - rest / a.NB;  // longest first
+  const int bl = a.b0 + rest % a.nblk;
+  const int p = a.SPB - 1 - rest / a.nblk;  // longest first
   it.b = bl;
   const int len = a.tb.blk_len[bl];
   if (p * 128 >= len) return it;
@@ -575,7 +636,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const int n_routed = *a.n_routed;
-  const int n_items = 2 * n_routed + a.H * a.NB * a.SPB;
+  const int n_items = 2 * n_routed + a.H * a.nblk * a.SPB;
   const uint64_t TO = a.wait_ns;
   int* err = a.status;
   auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -598,7 +659,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int e = 0; e < 4; ++e) {
         const int m = 4 * lane + e;
         const int mm = m < it.rows ? m : 0;  // padding rows repeat row 0 (never written)
-        rows4[e] = it.kind == 1 ? __ldg(a.entries + it.start + mm) / a.topk
+        rows4[e] = it.kind == 1 ? a.T0 * a.H + __ldg(a.entries + it.start + mm) / a.topk
                                 : (it.start + mm) * a.H + it.h;
       }
       if (lane == 0) mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE);
@@ -711,7 +772,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int row = 0, t = 0;
       if (rvalid) {
         if (it.kind == 1) {
-          row = __ldg(a.entries + it.start + m) / a.topk;
+          row = a.T0 * a.H + __ldg(a.entries + it.start + m) / a.topk;
           t = row / a.H;
         } else {
           t = it.start + m;
@@ -722,38 +783,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                       1.4426950408889634f
                                 : INFINITY;
       const float dsv = rvalid ? __ldg(a.dsum + row) : 0.f;
-      const int tlim = (it.kind == 2) ? t : 0x7fffffff;  // causal inside the query's own block
       for (int j = 0; j < it.nsub; ++j, ++cs) {
         ok = wait_all(&bars->s_full, cs & 1);
         if (!ok) break;
         tc_fence_after();
         const int u0 = it.key0 + j * 128;
-        const int kmax = min(it.klen - j * 128, 128);  // valid key columns of the sub-tile
-#pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-          uint32_t sr[32], dr[32];
-          tmem_ld32(tmem + lane_off + TM_S + c0, sr);
-          tmem_ld32(tmem + lane_off + TM_DP + c0, dr);
-          tmem_wait_ld();
+        // valid key columns: inside the block, and (own block) not after the query
+        int kmax = min(it.klen - j * 128, 128);
+        if (it.kind == 2) kmax = min(kmax, t - u0 + 1);
+        uint32_t sr[2][32], dr[2][32];
+        tmem_ld32(tmem + lane_off + TM_S, sr[0]);
+        tmem_ld32(tmem + lane_off + TM_DP, dr[0]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const int cur = ch & 1;
+          if (ch < 3) {
+            tmem_ld32(tmem + lane_off + TM_S + 32 * (ch + 1), sr[cur ^ 1]);
+            tmem_ld32(tmem + lane_off + TM_DP + 32 * (ch + 1), dr[cur ^ 1]);
+          }
 #pragma unroll
           for (int x = 0; x < 32; ++x) {
-            reg_fence(sr[x]);
-            reg_fence(dr[x]);
+            reg_fence(sr[cur][x]);
+            reg_fence(dr[cur][x]);
           }
           uint32_t dd[16];
 #pragma unroll
           for (int x = 0; x < 32; x += 2) {
-            float ds[2];
-#pragma unroll
-            for (int y = 0; y < 2; ++y) {
-              const int c = c0 + x + y;
-              const bool on = c < kmax && u0 + c <= tlim;
-              const float p = on ? ex2_approx(fmaf(__uint_as_float(sr[x + y]), sl2, -lse2)) : 0.f;
-              ds[y] = p * (__uint_as_float(dr[x + y]) - dsv);
-            }
-            dd[x >> 1] = pack_bf16x2(ds[0], ds[1]);
+            const int c = 32 * ch + x;
+            const float p0 = c < kmax ? ex2_approx(fmaf(__uint_as_float(sr[cur][x]), sl2, -lse2))
+                                      : 0.f;
+            const float p1 = c + 1 < kmax
+                                 ? ex2_approx(fmaf(__uint_as_float(sr[cur][x + 1]), sl2, -lse2))
+                                 : 0.f;
+            dd[x >> 1] = pack_bf16x2(p0 * (__uint_as_float(dr[cur][x]) - dsv),
+                                     p1 * (__uint_as_float(dr[cur][x + 1]) - dsv));
           }
-          tmem_st16(tmem + lane_off + TM_DP + c0 / 2, dd);
+          tmem_st16(tmem + lane_off + TM_DP + 16 * ch, dd);
+          if (ch < 3) tmem_wait_ld();
         }
         tmem_wait_st();
         tc_fence_before();
@@ -801,10 +868,13 @@ static BwdArgs bwd_args(const BwdLaunch& L) {
   a.bucket_end = L.bucket_end;
   a.tiles = L.tiles;
   a.n_routed = L.n_routed;
+  a.col_lse = L.col_lse;
+  a.col_d = L.col_d;
+  a.col_t = L.col_t;
   a.tb = L.tb;
-  a.dk = static_cast<__nv_bfloat16*>(L.dk);
-  a.dv = static_cast<__nv_bfloat16*>(L.dv);
   a.dq_acc = L.dq_acc;
+  a.dk_acc = L.dk_acc;
+  a.dv_acc = L.dv_acc;
   a.status = L.status;
   a.T = L.T;
   a.H = L.H;
@@ -813,17 +883,32 @@ static BwdArgs bwd_args(const BwdLaunch& L) {
   a.topk = L.topk;
   a.NB = L.NB;
   a.SPB = (L.B + 127) / 128;
+  a.T0 = L.T0;
+  a.b0 = L.b0;
+  a.nblk = L.nblk;
   a.scale = L.scale;
   a.scale_log2 = L.scale * 1.4426950408889634f;
   a.wait_ns = L.wait_ns > 0 ? L.wait_ns : kWaitTimeoutNs;
   return a;
 }
 
-static bool bwd_maps(const BwdLaunch& L, CUtensorMap* mk, CUtensorMap* mv, CUtensorMap* mq,
-                     CUtensorMap* mdo) {
-  return make_kv_map(mk, L.k, L.T, L.G, L.d) && make_kv_map(mv, L.v, L.T, L.G, L.d) &&
-         make_q_rows_map(mq, L.q, static_cast<long long>(L.T) * L.H, L.d) &&
-         make_q_rows_map(mdo, L.dout, static_cast<long long>(L.T) * L.H, L.d);
+// [rows, D] bf16 dense rows -> 2-D map (D, rows), box (64, 128), 128-byte swizzle, zero fill past
+// the last row.
+static bool make_rows_tile_map(CUtensorMap* map, const void* base, long long rows, int D) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t es[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static unsigned grid_for(long long n, int per_block, int num_sms) {
+  return static_cast<unsigned>(
+      std::max<long long>(1, std::min<long long>((n + per_block - 1) / per_block, 8LL * num_sms)));
 }
 
 cudaError_t launch_bwd_pre(const BwdLaunch& L, cudaStream_t stream) {
@@ -835,13 +920,41 @@ cudaError_t launch_bwd_pre(const BwdLaunch& L, cudaStream_t stream) {
     bwd_pre_kernel<64><<<grid, 256, 0, stream>>>(o, dout, rows, L.dsum, L.dq_acc);
   else
     bwd_pre_kernel<128><<<grid, 256, 0, stream>>>(o, dout, rows, L.dsum, L.dq_acc);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long n4 = static_cast<long long>(L.T) * L.G * L.d / 4;
+  bwd_zero_kernel<<<grid_for(n4, 256, L.num_sms), 256, 0, stream>>>(
+      reinterpret_cast<float4*>(L.dk_acc), n4);
+  bwd_zero_kernel<<<grid_for(n4, 256, L.num_sms), 256, 0, stream>>>(
+      reinterpret_cast<float4*>(L.dv_acc), n4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_densify(const BwdLaunch& L, cudaStream_t stream) {
+  const auto* q = static_cast<const __nv_bfloat16*>(L.q);
+  const auto* dout = static_cast<const __nv_bfloat16*>(L.dout);
+  auto* qd = static_cast<__nv_bfloat16*>(L.qd);
+  auto* dd = static_cast<__nv_bfloat16*>(L.dd);
+  const unsigned grid = grid_for(L.dense_rows, 256 / (L.d / 8), L.num_sms);
+  if (L.d == 64)
+    bwd_densify_kernel<64><<<grid, 256, 0, stream>>>(L.entries, L.n_routed + 1, q, dout, L.lse,
+                                                     L.dsum, L.T, L.H, L.topk, L.T0, qd, dd,
+                                                     L.col_lse, L.col_d, L.col_t);
+  else
+    bwd_densify_kernel<128><<<grid, 256, 0, stream>>>(L.entries, L.n_routed + 1, q, dout, L.lse,
+                                                      L.dsum, L.T, L.H, L.topk, L.T0, qd, dd,
+                                                      L.col_lse, L.col_d, L.col_t);
   return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t launch_dkdv_d(const BwdLaunch& L, cudaStream_t stream) {
-  CUtensorMap mk, mv, mq, mdo;
-  if (!bwd_maps(L, &mk, &mv, &mq, &mdo)) return cudaErrorInvalidValue;
+  CUtensorMap mk, mv, mq3, mdo3, mqd, mdd;
+  if (!make_kv_map(&mk, L.k, L.T, L.G, D) || !make_kv_map(&mv, L.v, L.T, L.G, D) ||
+      !make_kv_map(&mq3, L.q, L.T, L.H, D) || !make_kv_map(&mdo3, L.dout, L.T, L.H, D) ||
+      !make_rows_tile_map(&mqd, L.qd, std::max(L.dense_rows, 1LL), D) ||
+      !make_rows_tile_map(&mdd, L.dd, std::max(L.dense_rows, 1LL), D))
+    return cudaErrorInvalidValue;
   const BwdArgs a = bwd_args(L);
   const int n_kv = a.NB * a.G * a.SPB;
   // each CTA allocates all 512 tensor-memory columns: ask for enough shared memory that two CTAs
@@ -851,14 +964,17 @@ static cudaError_t launch_dkdv_d(const BwdLaunch& L, cudaStream_t stream) {
       cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   bwd_dkdv_kernel<D><<<std::min(L.num_sms, std::max(n_kv, 1)), kBwdThreads, smem, stream>>>(
-      mk, mv, mq, mdo, a, n_kv);
+      mk, mv, mq3, mdo3, mqd, mdd, a, n_kv);
   return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t launch_dq_d(const BwdLaunch& L, cudaStream_t stream) {
   CUtensorMap mk, mv, mq, mdo;
-  if (!bwd_maps(L, &mk, &mv, &mq, &mdo)) return cudaErrorInvalidValue;
+  if (!make_kv_map(&mk, L.k, L.T, L.G, D) || !make_kv_map(&mv, L.v, L.T, L.G, D) ||
+      !make_q_rows_map(&mq, L.q, static_cast<long long>(L.T) * L.H, D) ||
+      !make_q_rows_map(&mdo, L.dout, static_cast<long long>(L.T) * L.H, D))
+    return cudaErrorInvalidValue;
   const BwdArgs a = bwd_args(L);
   const int smem = std::max(QCfg<D>::SMEM, kOneCtaPerSmBytes);
   cudaError_t e =
@@ -877,12 +993,14 @@ cudaError_t launch_bwd_dq(const BwdLaunch& L, cudaStream_t stream) {
 }
 
 cudaError_t launch_bwd_finish(const BwdLaunch& L, cudaStream_t stream) {
-  const long long n4 = static_cast<long long>(L.T) * L.H * L.d / 4;
-  const unsigned grid =
-      static_cast<unsigned>(std::min<long long>((n4 + 255) / 256, 8LL * L.num_sms));
-  if (grid == 0) return cudaSuccess;
-  bwd_dq_finish_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(L.dq_acc), n4,
-                                                 static_cast<uint2*>(L.dq));
+  const long long nq4 = static_cast<long long>(L.T) * L.H * L.d / 4;
+  const long long nk4 = static_cast<long long>(L.T) * L.G * L.d / 4;
+  bwd_finish_kernel<<<grid_for(nq4, 256, L.num_sms), 256, 0, stream>>>(
+      reinterpret_cast<const float4*>(L.dq_acc), nq4, static_cast<uint2*>(L.dq));
+  bwd_finish_kernel<<<grid_for(nk4, 256, L.num_sms), 256, 0, stream>>>(
+      reinterpret_cast<const float4*>(L.dk_acc), nk4, static_cast<uint2*>(L.dk));
+  bwd_finish_kernel<<<grid_for(nk4, 256, L.num_sms), 256, 0, stream>>>(
+      reinterpret_cast<const float4*>(L.dv_acc), nk4, static_cast<uint2*>(L.dv));
   return cudaGetLastError();
 }
 

@@ -124,26 +124,36 @@ struct DecodeLaunch {
 int decode_parts(int B, int topk);
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream);
 
-// Backward pass of the routed attention (csrc/attn_bwd.cu).
+// Backward pass of the routed attention (csrc/attn_bwd.cu), one query chunk at a time.
 struct BwdLaunch {
   const void *q, *k, *v, *o, *dout;  // bf16 [T, H or G, d]
   const float* lse;                  // [H, T]
-  const int* entries;                // routed entries grouped by (g, b) (routing inversion)
+  const int* entries;                // chunk's routed entries grouped by (g, b)
   const int* bucket_end;             // [G * NB] end of every list after the scatter
   const int4* tiles;                 // routed 256-row items
-  const int* n_routed;
+  const int* n_routed;               // [0] routed items, [1] routed entries of the chunk
   BlockTables tb;
   float* dsum;                       // [T * H] scratch: D = dO . O
-  float* dq_acc;                     // [T * H, d] scratch: fp32 dQ accumulator
+  float* dq_acc;                     // [T * H, d] fp32 accumulators
+  float* dk_acc;                     // [T * G, d]
+  float* dv_acc;
+  void* qd;                          // [dense_rows, d] densified query rows of the chunk
+  void* dd;                          // [dense_rows, d] densified dO rows
+  float* col_lse;                    // [dense_rows] log2-domain LSE, D, position per dense row
+  float* col_d;
+  int* col_t;
+  long long dense_rows;              // capacity of the dense arrays (max entries of a chunk)
   void *dq, *dk, *dv;                // bf16 outputs
   int* status;
   int T, H, G, d, B, topk, NB, num_sms;
+  int T0, b0, nblk;                  // the chunk
   float scale;
   unsigned long long wait_ns = 0;
 };
-// D = dO . O and the zeroed dQ accumulator; the key-stationary dK / dV kernel; the
-// query-stationary dQ kernel; dQ converted to bf16.
+// Once: D = dO . O and the zeroed accumulators. Per chunk: densify the routed rows, the
+// key-stationary dK / dV kernel, the query-stationary dQ kernel. Once: bf16 outputs.
 cudaError_t launch_bwd_pre(const BwdLaunch& L, cudaStream_t stream);
+cudaError_t launch_bwd_densify(const BwdLaunch& L, cudaStream_t stream);
 cudaError_t launch_bwd_dkdv(const BwdLaunch& L, cudaStream_t stream);
 cudaError_t launch_bwd_dq(const BwdLaunch& L, cudaStream_t stream);
 cudaError_t launch_bwd_finish(const BwdLaunch& L, cudaStream_t stream);

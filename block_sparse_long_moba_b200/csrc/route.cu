@@ -84,8 +84,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
 // n = min(topk, i + 1), slots 0 .. n-2 hold strictly ascending past blocks (0 <= j < i), slot n-1
 // holds the current block i and the remaining slots hold -1. The diagonal tiles write slot n-1
 // and the merge reads slots 0 .. n-1, so a row that breaks this (e.g. a caller-supplied routing
-// with fewer blocks) would merge slots nobody wrote: it is reported as kDevBadRouting. Entries
-// outside 0 <= j < i are never counted or scattered, so a bad row cannot index out of bounds.
+// with fewer blocks) would merge slots nobody wrote: it is reported as kDevBadRouting. Only slots
+// 0 .. n-2 holding 0 <= j < i are counted and scattered, so a bad row can neither index out of
+// bounds nor add more than n - 1 entries (the lists are sized for exactly that many per row).
 template <bool kScatter>
 __global__ void __launch_bounds__(256) route_pass_kernel(
     const int32_t* __restrict__ idx, BlockTables tb, int T, int H, int G, int topk, int NB,
@@ -114,7 +115,7 @@ __global__ void __launch_bounds__(256) route_pass_kernel(
         bad |= slot < n - 1 ? (j <= prev || j >= i) : slot == n - 1 ? (j != i) : (j != -1);
         prev = j;
       }
-      if (j >= 0 && j < i) atomicAdd(&hist[j], 1);
+      if (slot < n - 1 && j >= 0 && j < i) atomicAdd(&hist[j], 1);
     }
   }
   if (!kScatter) {
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(256) route_pass_kernel(
     const int h = g * r + hh;
     const int32_t* rp = idx + (static_cast<size_t>(h) * T + t) * topk;
     const int prow = ((t - T0) * H + h) * topk;
-    for (int slot = 0; slot < topk; ++slot) {
+    for (int slot = 0; slot < n - 1; ++slot) {
       const int j = __ldg(rp + slot);
       if (j >= 0 && j < i) {
         const int pos = atomicAdd(&hist[j], 1);
