@@ -177,7 +177,7 @@ int make_plan(int nseq, const int32_t* cu, int Hq, int Hkv, int d, int B, int to
 
 // --------------------------------------------------------------------------- workspace carve
 struct Layout {
-  size_t status, blk_off, blk_seq, blk_start, blk_len, cents, idx, counts, cursor, tiles,
+  size_t status, blk_off, blk_seq, blk_start, blk_len, cents, split, idx, counts, cursor, tiles,
       entries, qdense, part_o, part_lse, total;
 };
 
@@ -193,6 +193,7 @@ Layout layout_of(const Plan& P, int nseq, int Hq, int Hkv, int d, int topk) {
   L.blk_start = take(static_cast<size_t>(P.NB) * 4);
   L.blk_len = take(static_cast<size_t>(P.NB) * 4);
   L.cents = take(static_cast<size_t>(P.NB) * Hkv * d * 4);
+  L.split = take(gate_split_bytes(P.NB, Hkv, d));
   L.idx = take(static_cast<size_t>(Hq) * P.T * topk * 4);
   L.counts = take(static_cast<size_t>(Hkv) * P.NB * 4);
   L.cursor = take(static_cast<size_t>(Hkv) * P.NB * 4);
@@ -213,12 +214,14 @@ T* at(void* base, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(b
 // streaming gate (all past centroids resident, query tiles streamed by a producer warp).
 cudaError_t run_gate(const void* q, const float* cents, const int32_t* cu_dev,
                      const int32_t* cu_host, int nseq, int max_nb, int T, int H, int G, int d,
-                     int B, int topk, int32_t* idx, int* status, int sms, cudaStream_t s) {
+                     int B, int topk, int32_t* idx, int* status, int sms, cudaStream_t s,
+                     const BlockTables* tb = nullptr, int NB = 0, void* split = nullptr) {
   if (gate_stream_supported(max_nb, topk))
     return launch_gate_stream(q, cents, cu_dev, cu_host, nseq, max_nb, T, H, G, d, B, topk, idx,
                               status, sms, s);
   if (topk <= 33)
-    return launch_gate_tc(q, cents, cu_dev, nseq, max_nb, T, H, G, d, B, topk, idx, status, sms, s);
+    return launch_gate_tc(q, cents, cu_dev, nseq, max_nb, T, H, G, d, B, topk, idx, status, sms, s,
+                          tb, NB, split);
   return launch_gate(q, cents, cu_dev, nseq, max_nb, T, H, G, d, B, topk, idx, s);
 }
 
@@ -381,7 +384,7 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu
                                  conv_w, conv_width));
     MOBA_LAUNCH(kGate, s,
                 run_gate(q, cents, cu_dev, cu_host, nseq, P.max_nb, P.T, Hq, Hkv, d, block_size,
-                         topk, idx_w, status, sms, s));
+                         topk, idx_w, status, sms, s, &tb, P.NB, at<void>(workspace, L.split)));
     idx = idx_w;
   } else if (block_idx_out && block_idx_out != block_idx_in) {
     if (cudaMemcpyAsync(block_idx_out, block_idx_in, static_cast<size_t>(Hq) * P.T * topk * 4,

@@ -10,23 +10,25 @@
 // FlashTopK]: at most 256 scores per row at a time live in tensor memory, and the products are
 // recomputed for each pass below (the tensor pipe is otherwise idle here).
 //
-// Selection, one thread per row (= TMEM lane), in three passes over the row's n scores:
+// Selection, one thread per row (= TMEM lane), in two passes over the row's n scores:
 //   1. group maxima over M strided groups (column j in group j mod M, M = 32 or 64); the ksel-th
 //      largest group maximum tau is a lower bound of the ksel-th best score, since ksel distinct
 //      groups each hold a score >= tau;
-//   2. every score >= tau is a candidate (typically ksel + a few) and is appended to the row's
-//      candidate buffer in shared memory; a bitonic sort of the buffer gives the exact ksel-th
-//      best score tau* and how many of the selected scores tie with it;
-//   3. the columns with score > tau*, and the lowest-numbered ones equal to tau* (ties go to the
-//      lower block), are written out in ascending order.
-// Each pass costs a compare per score and no per-score list insertion; a single pass that keeps a
-// running top list pays an insertion for every score that beats the list's current threshold,
-// which is most of the early columns. A row whose candidates overflow the buffer (many exactly
-// equal scores) runs that single-pass selection in pass 3 instead.
+//   2. every score >= tau is a candidate (typically ksel + a few) and is appended, with its block,
+//      to the row's candidate buffer in shared memory (in ascending block order); a bitonic sort
+//      of the candidate scores gives the exact ksel-th best score tau* and how many selected
+//      scores tie with it, and a walk over the buffer writes the blocks with score > tau* and the
+//      lowest-numbered ones equal to tau* (ties go to the lower block), already ascending.
+// Each pass costs a compare per score and no per-score list insertion. A row whose candidates
+// overflow the buffer (many exactly equal scores) runs a third pass with a running top list.
 //
 // A CTA holds two warpgroups (one query tile each) and works on one (query blocks, kv head) unit
-// at a time: the split centroids of the unit's past blocks are converted into shared memory once
-// and reused by all tiles of the unit when they fit, and streamed in chunks otherwise.
+// at a time: the hi / lo centroids of the unit's past blocks are placed in shared memory once and
+// reused by all tiles of the unit when they fit, and streamed in chunks otherwise. Inside the
+// forward pass they come pre-split from global memory (one bulk copy per chunk and part, in the
+// swizzled row layout the MMA reads); the standalone gate converts the fp32 centroids itself.
+#include <algorithm>
+
 #include "common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
@@ -43,9 +45,9 @@ struct GateCfg {
   static constexpr int M = (KCAP <= 16) ? 32 : 64;           // groups of pass 1
   static constexpr int CB = (KCAP <= 16) ? 32 : 64;          // candidate slots per row
   static constexpr int Q_BYTES = kTile * D * 2;             // one 128-row query tile
-  static constexpr int CAND_BYTES = 2 * CB * 128 * 4;        // [2][CB][128] fp32
-  // centroid rows resident at once: what is left of the CTA's shared memory
-  static constexpr int CAP = (D == 128) ? (KCAP <= 16 ? 256 : 192) : (KCAP <= 16 ? 640 : 512);
+  static constexpr int CAND_BYTES = 2 * CB * 128 * 8;        // [2][CB][128] fp32 + [2][CB][128] int
+  // centroid rows resident at once (a multiple of 16): what is left of the CTA's shared memory
+  static constexpr int CAP = (D == 128) ? (KCAP <= 16 ? 192 : 64) : (KCAP <= 16 ? 512 : 256);
   static constexpr int B_BYTES = 2 * NCB * CAP * 128;        // hi + lo, 128 B per row per block
   static constexpr int OFF_B = 2 * Q_BYTES;                  // one Q buffer per warpgroup
   static constexpr int OFF_STAGE = OFF_B + B_BYTES;          // candidate buffer / staging
@@ -58,7 +60,7 @@ static_assert(GateCfg<128, 16>::SMEM_BYTES <= 232448 && GateCfg<64, 16>::SMEM_BY
               "shared memory budget of one CTA");
 
 struct GateBars {
-  uint64_t q_full[2], mma_done[2][2];
+  uint64_t q_full[2], mma_done[2][2], chunk_full;
   uint32_t tmem_base;
   int abort_flag;
   int red[32];
@@ -146,7 +148,8 @@ template <int D, int KCAP>
 __global__ void __launch_bounds__(256, 1)
     gate_tc_kernel(const __grid_constant__ CUtensorMap map_q, const float* __restrict__ cents,
                    const int32_t* __restrict__ cu, int nseq, int max_nb, int T, int H, int G,
-                   int B, int topk, int32_t* __restrict__ idx, int* __restrict__ status) {
+                   int B, int topk, int32_t* __restrict__ idx, int* __restrict__ status,
+                   const uint8_t* __restrict__ split, int nb_pad) {
   using C = GateCfg<D, KCAP>;
   constexpr int M = C::M, CB = C::CB;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -164,6 +167,7 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(&bars->mma_done[x][0], 1);
       mbar_init(&bars->mma_done[x][1], 1);
     }
+    mbar_init(&bars->chunk_full, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -178,8 +182,12 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t tmem = bars->tmem_base;
   const uint32_t t_s = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + wg * 2 * C::PIECE;
   uint8_t* sQ = smem + wg * C::Q_BYTES;
-  // this warpgroup's candidate buffer [CB][128] (pass 2), reused as staging [32][128] (pass 3)
+  // this warpgroup's candidate buffer [CB][128] scores + [CB][128] blocks (pass 2), the scores
+  // part reused as staging [32][128] (pass 3)
   float* cand = reinterpret_cast<float*>(smem + C::OFF_STAGE) + wg * CB * 128;
+  int* candi = reinterpret_cast<int*>(smem + C::OFF_STAGE) + 2 * CB * 128 + wg * CB * 128;
+  uint32_t chunk_phase = 0;   // chunk_full phase (pre-split centroids)
+  bool chunk_pending = false; // a chunk copy issued by thread 0 that no wait has seen land
   const uint32_t sBa = smem_u32(smem + C::OFF_B);
   const int r = H / G;
   const int ksel = topk - 1;
@@ -282,10 +290,35 @@ __global__ void __launch_bounds__(256, 1)
       top.init(ksel);
       bool q_ready = false;
       for (int pass = 0; pass < 3; ++pass) {
+        // the third pass only runs for rows whose candidates overflowed (CTA-uniform decision)
+        if (pass == 2 && !__syncthreads_or(overflow && scored && row < rows)) break;
         for (int ch = 0; ch < nchunks; ++ch) {
           const int c0 = ch * C::CAP;
           const int n = min(C::CAP, i_max - c0);
-          if (nchunks > 1 || (p == 0 && pass == 0)) {
+          if ((nchunks > 1 || (p == 0 && pass == 0)) && split) {
+            // pre-split hi / lo rows of blocks [c0, c0 + n) (16-row padded): one bulk copy per
+            // part and 64-column atom; rows were swizzled by their block's index in its sequence,
+            // and c0 % 8 == 0, so they land in the layout the MMA reads
+            ok = __syncthreads_and(ok);
+            const int rows_pad = (n + 15) & ~15;
+            if (tid == 0 && ok) {
+              mbar_arrive_expect_tx(&bars->chunk_full, 2 * C::NCB * rows_pad * 128);
+#pragma unroll
+              for (int part = 0; part < 2; ++part)
+#pragma unroll
+                for (int at = 0; at < C::NCB; ++at)
+                  bulk_load(smem + C::OFF_B + c_offset<D, KCAP>(part, 0, 64 * at),
+                            split + ((static_cast<size_t>(g * 2 + part) * C::NCB + at) * nb_pad +
+                                     base + c0) * 128,
+                            rows_pad * 128, &bars->chunk_full);
+              chunk_pending = true;
+            }
+            const bool w = ok && mbar_wait_bounded(&bars->chunk_full, chunk_phase, abort_flag,
+                                                   status, kDevTimeoutAttn, TO);
+            chunk_phase ^= 1;
+            if (tid == 0 && w) chunk_pending = false;
+            ok = __syncthreads_and(w);
+          } else if (nchunks > 1 || (p == 0 && pass == 0)) {
             // split the fp32 centroids of blocks [c0, c0 + n) into hi / lo bf16 tiles; each thread
             // issues the loads of eight 8-column groups before converting any
             ok = __syncthreads_and(ok);
@@ -379,13 +412,6 @@ __global__ void __launch_bounds__(256, 1)
             }
             const bool w = ok && mbar_wait_bounded(&bars->mma_done[wg][pc & 1], (pc >> 1) & 1,
                                                    abort_flag, status, kDevTimeoutAttn, TO);
-            // the Q buffer is free once the tile's last product of the last pass is done
-            const bool last_pass = pass == 2 && (c0 + n >= i_t || ch == nchunks - 1) &&
-                                   p0 + C::PIECE >= n_t;
-            if (row == 0 && w && last_pass) {
-              const int t = next_scored(tile + 2);
-              if (t < ntiles) load_q(t);
-            }
             if (__all_sync(0xffffffffu, w)) {
               tc_fence_after();
               const uint32_t tb = t_s + (pc & 1) * C::PIECE;
@@ -409,37 +435,19 @@ __global__ void __launch_bounds__(256, 1)
                         gmax[(32 + x) % M] = fmaxf(gmax[(32 + x) % M], __uint_as_float(sr[x]));
                   }
                 } else if (pass == 1) {
-                  // every score >= tau is a candidate
+                  // every score >= tau is a candidate, kept with its block (ascending)
 #pragma unroll
                   for (int x = 0; x < 32; ++x) {
                     const float sv = __uint_as_float(sr[x]);
                     if (cc + x < np && sv >= tau) {
-                      if (cnt < CB) cand[cnt * 128 + row] = sv;
+                      if (cnt < CB) {
+                        cand[cnt * 128 + row] = sv;
+                        candi[cnt * 128 + row] = jb + x;
+                      }
                       ++cnt;
                     }
                   }
                 } else {
-                  if (!overflow) {
-                    // columns above tau*, and the lowest-numbered ties while the budget lasts
-                    uint32_t gtm = 0, eqm = 0;
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) {
-                      const float sv = __uint_as_float(sr[x]);
-                      if (cc + x < np) {
-                        if (sv > tau_star) gtm |= 1u << x;
-                        else if (sv == tau_star) eqm |= 1u << x;
-                      }
-                    }
-                    while (__popc(eqm) > tie_budget) eqm &= ~(1u << (31 - __clz(eqm)));
-                    tie_budget -= __popc(eqm);
-                    uint32_t m = gtm | eqm;
-                    while (m) {
-                      const int x = __ffs(m) - 1;
-                      m &= m - 1;
-                      if (row < rows) out[pos] = jb + x;
-                      ++pos;
-                    }
-                  }
                   // rows whose candidates overflowed keep a running top list instead
                   const float thr0 = top.thr();
                   uint32_t mask = 0;
@@ -487,8 +495,21 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
             for (int x = 0; x < CB; ++x) above += (cv[x] > tau_star) ? 1 : 0;
             tie_budget = ksel - above;
+            // the buffer is in ascending block order: blocks above tau*, then the lowest ties
+            for (int x = 0; x < cnt; ++x) {
+              const float sv = cand[x * 128 + row];
+              if (sv > tau_star || (sv == tau_star && tie_budget-- > 0)) {
+                if (row < rows) out[pos] = candi[x * 128 + row];
+                ++pos;
+              }
+            }
           }
         }
+      }
+      // the Q buffer is free: every product of this tile is done; load the next scored tile
+      if (scored && row == 0 && ok) {
+        const int t = next_scored(tile + 2);
+        if (t < ntiles) load_q(t);
       }
       if (!scored || row >= rows || !ok) continue;
       if (overflow) {
@@ -514,11 +535,68 @@ __global__ void __launch_bounds__(256, 1)
     ok = __syncthreads_and(ok);
     if (!ok) break;
   }
+  if (tid == 0 && chunk_pending) {
+    // a chunk copy whose landing no wait saw: let it land before the CTA exits (bounded)
+    volatile int no_abort = 0;
+    mbar_wait_bounded(&bars->chunk_full, chunk_phase ^ 1, &no_abort, status, kDevDrainTimeout,
+                      kDrainTimeoutNs);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// Pre-split centroids for the gate: for kv head g, part (0 = hi, 1 = lo bf16 of the fp32
+// centroid), 64-column atom a and global block b, one 128-byte row at
+// (((g * 2 + part) * NCB + a) * nb_pad + b) * 128 with its 16-byte pieces swizzled by the
+// block's index inside its sequence (mod 8) — the rows of a chunk that starts at a multiple of 8
+// then land in shared memory in the MMA's 128-byte-swizzle layout. Rows b >= NB are zero.
+template <int D>
+__global__ void __launch_bounds__(256) split_cents_kernel(const float* __restrict__ cents,
+                                                          BlockTables tb, int NB, int nb_pad,
+                                                          int G, uint8_t* __restrict__ split) {
+  constexpr int NCB = D / 64;
+  const long long n = static_cast<long long>(nb_pad) * G * NCB * 8;  // 16-byte pieces per part
+  for (long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; x < n;
+       x += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(x % 8);
+    long long rest = x / 8;
+    const int at = static_cast<int>(rest % NCB);
+    rest /= NCB;
+    const int b = static_cast<int>(rest % nb_pad);
+    const int g = static_cast<int>(rest / nb_pad);
+    uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
+    int j = 0;
+    if (b < NB) {
+      j = b - tb.blk_off[tb.blk_seq[b]];
+      const float4* src =
+          reinterpret_cast<const float4*>(cents + (static_cast<size_t>(b) * G + g) * D + at * 64 + c * 8);
+      const float4 va = __ldg(src), vb = __ldg(src + 1);
+      const float v[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * k]);
+        const __nv_bfloat16 h1 = __float2bfloat16_rn(v[2 * k + 1]);
+        const __nv_bfloat16 l0 = __float2bfloat16_rn(v[2 * k] - __bfloat162float(h0));
+        const __nv_bfloat16 l1 = __float2bfloat16_rn(v[2 * k + 1] - __bfloat162float(h1));
+        hw[k] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+        lw[k] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
+                (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+      }
+      hi = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      lo = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    const size_t piece = static_cast<size_t>((c ^ (j & 7)) & 7) * 16;
+    *reinterpret_cast<uint4*>(split + ((static_cast<size_t>(g * 2) * NCB + at) * nb_pad + b) * 128 +
+                              piece) = hi;
+    *reinterpret_cast<uint4*>(split + ((static_cast<size_t>(g * 2 + 1) * NCB + at) * nb_pad + b) *
+                                          128 +
+                              piece) = lo;
   }
 }
 
@@ -553,39 +631,71 @@ bool make_q_map(CUtensorMap* map, const void* q, int T, int H, int D) {
 template <int D, int KCAP>
 cudaError_t launch_t(const CUtensorMap& mq, const float* cents, const int32_t* cu, int nseq,
                      int max_nb, int T, int H, int G, int B, int topk, int32_t* idx, int* status,
-                     int grid, cudaStream_t stream) {
+                     int grid, cudaStream_t stream, const uint8_t* split, int nb_pad) {
   const int smem = GateCfg<D, KCAP>::SMEM_BYTES;
   cudaError_t e = cudaFuncSetAttribute(gate_tc_kernel<D, KCAP>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   gate_tc_kernel<D, KCAP><<<grid, 256, smem, stream>>>(mq, cents, cu, nseq, max_nb, T, H, G, B,
-                                                       topk, idx, status);
+                                                       topk, idx, status, split, nb_pad);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_d(const CUtensorMap& mq, const float* cents, const int32_t* cu, int nseq,
                      int max_nb, int T, int H, int G, int B, int topk, int32_t* idx, int* status,
-                     int grid, cudaStream_t stream) {
+                     int grid, cudaStream_t stream, const uint8_t* split, int nb_pad) {
   const int ksel = topk - 1;
-  if (ksel <= 4) return launch_t<D, 4>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status, grid, stream);
-  if (ksel <= 8) return launch_t<D, 8>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status, grid, stream);
-  if (ksel <= 16) return launch_t<D, 16>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status, grid, stream);
-  return launch_t<D, 32>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status, grid, stream);
+  if (ksel <= 4)
+    return launch_t<D, 4>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status, grid,
+                          stream, split, nb_pad);
+  if (ksel <= 8)
+    return launch_t<D, 8>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status, grid,
+                          stream, split, nb_pad);
+  if (ksel <= 16)
+    return launch_t<D, 16>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status, grid,
+                           stream, split, nb_pad);
+  return launch_t<D, 32>(mq, cents, cu, nseq, max_nb, T, H, G, B, topk, idx, status, grid, stream,
+                         split, nb_pad);
 }
 
 }  // namespace
 
 cudaError_t launch_gate_tc(const void* q, const float* cents, const int32_t* cu_dev, int nseq,
                            int max_nb, int T, int H, int G, int d, int B, int topk, int32_t* idx,
-                           int* status, int num_sms, cudaStream_t stream) {
+                           int* status, int num_sms, cudaStream_t stream, const BlockTables* tb,
+                           int NB, void* split) {
   if (topk - 1 > 32) return cudaErrorInvalidValue;
   CUtensorMap mq;
   if (!make_q_map(&mq, q, T, H, d)) return cudaErrorInvalidValue;
   const int grid = num_sms > 0 ? num_sms : 1;  // persistent CTAs over the work units
+  const int nb_pad = NB + 16;
+  const uint8_t* sp = nullptr;
+  if (split && tb) {
+    const long long pieces = static_cast<long long>(nb_pad) * G * (d / 64) * 8;
+    const unsigned g2 = static_cast<unsigned>(
+        std::max<long long>(1, std::min<long long>((pieces + 255) / 256, 8LL * grid)));
+    if (d == 64)
+      split_cents_kernel<64><<<g2, 256, 0, stream>>>(cents, *tb, NB, nb_pad, G,
+                                                     static_cast<uint8_t*>(split));
+    else
+      split_cents_kernel<128><<<g2, 256, 0, stream>>>(cents, *tb, NB, nb_pad, G,
+                                                      static_cast<uint8_t*>(split));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    sp = static_cast<const uint8_t*>(split);
+  }
   if (d == 64)
-    return launch_d<64>(mq, cents, cu_dev, nseq, max_nb, T, H, G, B, topk, idx, status, grid, stream);
-  return launch_d<128>(mq, cents, cu_dev, nseq, max_nb, T, H, G, B, topk, idx, status, grid, stream);
+    return launch_d<64>(mq, cents, cu_dev, nseq, max_nb, T, H, G, B, topk, idx, status, grid,
+                        stream, sp, nb_pad);
+  return launch_d<128>(mq, cents, cu_dev, nseq, max_nb, T, H, G, B, topk, idx, status, grid,
+                       stream, sp, nb_pad);
+}
+
+// Bytes of the pre-split centroid buffer launch_gate_tc fills (hi and lo bf16 per fp32 value,
+// 16 padding rows).
+size_t gate_split_bytes(int NB, int G, int d) {
+  return static_cast<size_t>(NB + 16) * G * d * 4;
 }
 
 }  // namespace moba

@@ -43,10 +43,14 @@ cudaError_t launch_gate_stream(const void* q, const float* cents, const int32_t*
                                int d, int B, int topk, int32_t* idx, int* status, int num_sms,
                                cudaStream_t stream);
 
-// Tensor-core gate (scores on tcgen05, top-k in registers). `status` may be null.
+// Tensor-core gate (scores on tcgen05, top-k in registers). `status` may be null. With `split`
+// (gate_split_bytes(NB, G, d) bytes) and the block tables, the centroids are split into hi / lo
+// bf16 once into that buffer and the kernel copies chunks of it; otherwise it converts them itself.
 cudaError_t launch_gate_tc(const void* q, const float* cents, const int32_t* cu_dev, int nseq,
                            int max_nb, int T, int H, int G, int d, int B, int topk, int32_t* idx,
-                           int* status, int num_sms, cudaStream_t stream);
+                           int* status, int num_sms, cudaStream_t stream,
+                           const BlockTables* tb = nullptr, int NB = 0, void* split = nullptr);
+size_t gate_split_bytes(int NB, int G, int d);
 
 // Counts the routed entries per (kv head, block) and checks every routing row of the chunk
 // against its contract (kDevBadRouting in *status on the first bad row).
