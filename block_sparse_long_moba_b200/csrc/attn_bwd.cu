@@ -31,9 +31,11 @@
 //                    and adds scale * dQ once per item into the fp32 accumulator (red.global.add;
 //                    a row collects one addition per selected block).
 //   bwd_finish       dQ, dK, dV = bf16(accumulators).
-// Warp roles (256 threads): warp 0 = TMA producer (tiles and, for the query tiles, the per-row
-// LSE / D / position columns), warp 1 = TMEM owner and MMA issuer, warps 4-7 = one thread per
-// tensor-memory lane (the elementwise softmax-gradient step and the epilogues). Every wait is
+// Warp roles: warp 0 = TMA producer (tiles and, for the query tiles, the per-row LSE / D
+// columns), warp 1 = TMEM owner and MMA issuer, then one thread per tensor-memory lane for the
+// elementwise softmax-gradient step and the epilogues: warps 4-7 and 8-11 (384 threads; each
+// warpgroup takes half of the tile's columns: query rows in the dK/dV kernel, keys in the dQ
+// kernel). Every wait is
 // bounded; on a timeout the CTA raises its abort flag, records a status code, lets its copies and
 // matrix products in flight finish (under the fixed drain limit) and returns. No TMA multicast.
 #include <algorithm>
@@ -44,7 +46,7 @@
 
 namespace moba {
 
-constexpr int kBwdThreads = 256;
+constexpr int kKvThreads = 384;  // dK/dV and dQ kernels: two elementwise warpgroups
 constexpr int kOneCtaPerSmBytes = 120 * 1024;  // more than half of an SM's shared memory
 
 struct BwdArgs {
@@ -207,7 +209,7 @@ struct KvBars {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kKvThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v,
                     const __grid_constant__ CUtensorMap map_q3,
@@ -232,9 +234,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&bars->qd_empty[s], 1);
     }
     mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->p_full, 128);
+    mbar_init(&bars->p_full, 256);
     mbar_init(&bars->acc_full, 1);
-    mbar_init(&bars->acc_free, 128);
+    mbar_init(&bars->acc_free, 256);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -392,14 +394,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         {
           const uint64_t bd = smem_desc_sw128(sD, 16384, 1024), bq = smem_desc_sw128(sQ, 16384, 1024);
+          // packed rows 0..63 sit in columns 0..31 (first warpgroup), rows 64..127 in columns
+          // 64..95 (second warpgroup): each half writes only columns it has read itself
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            mma_ts_elect(tmem + TM_DV, tmem + TM_S + ks * 8, desc_advance(bd, ks * 2048), IDESC_ACC,
-                         (n > 0 || ks > 0) ? 1u : 0u);
+            mma_ts_elect(tmem + TM_DV, tmem + TM_S + (ks >> 2) * 64 + (ks & 3) * 8,
+                         desc_advance(bd, ks * 2048), IDESC_ACC, (n > 0 || ks > 0) ? 1u : 0u);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            mma_ts_elect(tmem + TM_DK, tmem + TM_DP + ks * 8, desc_advance(bq, ks * 2048),
-                         IDESC_ACC, (n > 0 || ks > 0) ? 1u : 0u);
+            mma_ts_elect(tmem + TM_DK, tmem + TM_DP + (ks >> 2) * 64 + (ks & 3) * 8,
+                         desc_advance(bq, ks * 2048), IDESC_ACC, (n > 0 || ks > 0) ? 1u : 0u);
           mma_commit_elect(&bars->qd_empty[st]);
         }
       }
@@ -415,7 +419,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------- P, dS (thread = key) and dK, dV
-    const int row = tid - 128;  // tensor-memory lane = key of the sub-tile
+    // two warpgroups on the same keys: half hw takes the tile's query columns 64 hw .. 64 hw + 63
+    // and the d columns hw D/2 .. hw D/2 + D/2 - 1 of the epilogue
+    const int hw = (warp - 4) >> 2;
+    const int row = (warp & 3) * 32 + (tid & 31);  // tensor-memory lane = key of the sub-tile
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float sl2 = a.scale_log2;
     uint32_t gt = 0, li = 0;
@@ -438,18 +445,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         int cmin = 0;
         if (n >= it.nrt) cmin = u - (it.key0 + ((n - it.nrt) % it.ndt_head) * 128);
         if (!kvalid) cmin = 128;
-        // 32-column chunks; the next chunk's tensor-memory loads are in flight while this one is
-        // computed. Packed P / dS of chunk ch go to columns 16 ch .. 16 ch + 15, already read.
+        // this half's two 32-column chunks; the second chunk's tensor-memory loads are in flight
+        // while the first is computed. Packed P / dS of chunk ch of half hw go to columns
+        // 64 hw + 16 ch .. + 15, inside this half's own (already read) columns.
+        const int cbase = 64 * hw;
         uint32_t sr[2][32], dr[2][32];
-        tmem_ld32(tmem + lane_off + TM_S, sr[0]);
-        tmem_ld32(tmem + lane_off + TM_DP, dr[0]);
+        tmem_ld32(tmem + lane_off + TM_S + cbase, sr[0]);
+        tmem_ld32(tmem + lane_off + TM_DP + cbase, dr[0]);
         tmem_wait_ld();
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 0; ch < 2; ++ch) {
           const int cur = ch & 1;
-          if (ch < 3) {
-            tmem_ld32(tmem + lane_off + TM_S + 32 * (ch + 1), sr[cur ^ 1]);
-            tmem_ld32(tmem + lane_off + TM_DP + 32 * (ch + 1), dr[cur ^ 1]);
+          if (ch < 1) {
+            tmem_ld32(tmem + lane_off + TM_S + cbase + 32, sr[1]);
+            tmem_ld32(tmem + lane_off + TM_DP + cbase + 32, dr[1]);
           }
 #pragma unroll
           for (int x = 0; x < 32; ++x) {
@@ -459,7 +468,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           uint32_t pp[16], dd[16];
 #pragma unroll
           for (int x = 0; x < 32; x += 2) {
-            const int c = 32 * ch + x;
+            const int c = cbase + 32 * ch + x;
             const float4 cc = cl4[c >> 1];  // {lse2, D} of columns c and c + 1
             const float p0 = c >= cmin ? ex2_approx(fmaf(__uint_as_float(sr[cur][x]), sl2, -cc.x))
                                        : 0.f;
@@ -470,9 +479,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             dd[x >> 1] = pack_bf16x2(p0 * (__uint_as_float(dr[cur][x]) - cc.y),
                                      p1 * (__uint_as_float(dr[cur][x + 1]) - cc.w));
           }
-          tmem_st16(tmem + lane_off + TM_S + 16 * ch, pp);
-          tmem_st16(tmem + lane_off + TM_DP + 16 * ch, dd);
-          if (ch < 3) tmem_wait_ld();
+          tmem_st16(tmem + lane_off + TM_S + cbase + 16 * ch, pp);
+          tmem_st16(tmem + lane_off + TM_DP + cbase + 16 * ch, dd);
+          if (ch < 1) tmem_wait_ld();
         }
         tmem_wait_st();
         tc_fence_before();
@@ -486,7 +495,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       float* dka = a.dk_acc + (static_cast<size_t>(u) * a.G + it.g) * D;
       float* dva = a.dv_acc + (static_cast<size_t>(u) * a.G + it.g) * D;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = hw * (D / 2); c0 < (hw + 1) * (D / 2); c0 += 32) {
         uint32_t kr[32], vr[32];
         tmem_ld32(tmem + lane_off + TM_DK + c0, kr);
         tmem_ld32(tmem + lane_off + TM_DV + c0, vr);
@@ -592,7 +601,7 @@ struct QBars {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kKvThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v,
                   const __grid_constant__ CUtensorMap map_q,
@@ -614,9 +623,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&bars->kv_empty[s], 1);
     }
     mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->ds_full, 128);
+    mbar_init(&bars->ds_full, 256);
     mbar_init(&bars->dq_full, 1);
-    mbar_init(&bars->dq_free, 128);
+    mbar_init(&bars->dq_free, 256);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -744,8 +753,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const uint64_t bk = smem_desc_sw128(sK, 16384, 1024);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            mma_ts_elect(tmem + TM_DQ, tmem + TM_DP + ks * 8, desc_advance(bk, ks * 2048), IDESC_DQ,
-                         (j > 0 || ks > 0) ? 1u : 0u);
+            // packed keys 0..63 in columns 0..31 (first warpgroup), 64..127 in 64..95
+            mma_ts_elect(tmem + TM_DQ, tmem + TM_DP + (ks >> 2) * 64 + (ks & 3) * 8,
+                         desc_advance(bk, ks * 2048), IDESC_DQ, (j > 0 || ks > 0) ? 1u : 0u);
           mma_commit_elect(&bars->kv_empty[st]);
         }
       }
@@ -760,7 +770,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp >= 4) {
     // ----------------------------------------------------------- dS (thread = query row), dQ
-    const int m = tid - 128;
+    // two warpgroups on the same rows: half hw takes key columns 64 hw .. 64 hw + 63 and d
+    // columns hw D/2 .. hw D/2 + D/2 - 1 of the epilogue
+    const int hw = (warp - 4) >> 2;
+    const int m = (warp & 3) * 32 + (tid & 31);
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float sl2 = a.scale_log2;
     uint32_t li = 0, cs = 0;
@@ -791,16 +804,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // valid key columns: inside the block, and (own block) not after the query
         int kmax = min(it.klen - j * 128, 128);
         if (it.kind == 2) kmax = min(kmax, t - u0 + 1);
+        const int cbase = 64 * hw;
         uint32_t sr[2][32], dr[2][32];
-        tmem_ld32(tmem + lane_off + TM_S, sr[0]);
-        tmem_ld32(tmem + lane_off + TM_DP, dr[0]);
+        tmem_ld32(tmem + lane_off + TM_S + cbase, sr[0]);
+        tmem_ld32(tmem + lane_off + TM_DP + cbase, dr[0]);
         tmem_wait_ld();
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 0; ch < 2; ++ch) {
           const int cur = ch & 1;
-          if (ch < 3) {
-            tmem_ld32(tmem + lane_off + TM_S + 32 * (ch + 1), sr[cur ^ 1]);
-            tmem_ld32(tmem + lane_off + TM_DP + 32 * (ch + 1), dr[cur ^ 1]);
+          if (ch < 1) {
+            tmem_ld32(tmem + lane_off + TM_S + cbase + 32, sr[1]);
+            tmem_ld32(tmem + lane_off + TM_DP + cbase + 32, dr[1]);
           }
 #pragma unroll
           for (int x = 0; x < 32; ++x) {
@@ -810,7 +824,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           uint32_t dd[16];
 #pragma unroll
           for (int x = 0; x < 32; x += 2) {
-            const int c = 32 * ch + x;
+            const int c = cbase + 32 * ch + x;
             const float p0 = c < kmax ? ex2_approx(fmaf(__uint_as_float(sr[cur][x]), sl2, -lse2))
                                       : 0.f;
             const float p1 = c + 1 < kmax
@@ -819,8 +833,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             dd[x >> 1] = pack_bf16x2(p0 * (__uint_as_float(dr[cur][x]) - dsv),
                                      p1 * (__uint_as_float(dr[cur][x + 1]) - dsv));
           }
-          tmem_st16(tmem + lane_off + TM_DP + 16 * ch, dd);
-          if (ch < 3) tmem_wait_ld();
+          tmem_st16(tmem + lane_off + TM_DP + cbase + 16 * ch, dd);
+          if (ch < 1) tmem_wait_ld();
         }
         tmem_wait_st();
         tc_fence_before();
@@ -832,7 +846,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       float* dst = a.dq_acc + static_cast<size_t>(row) * D;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = hw * (D / 2); c0 < (hw + 1) * (D / 2); c0 += 32) {
         uint32_t qr[32];
         tmem_ld32(tmem + lane_off + TM_DQ + c0, qr);
         tmem_wait_ld();
@@ -963,7 +977,7 @@ static cudaError_t launch_dkdv_d(const BwdLaunch& L, cudaStream_t stream) {
   cudaError_t e =
       cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  bwd_dkdv_kernel<D><<<std::min(L.num_sms, std::max(n_kv, 1)), kBwdThreads, smem, stream>>>(
+  bwd_dkdv_kernel<D><<<std::min(L.num_sms, std::max(n_kv, 1)), kKvThreads, smem, stream>>>(
       mk, mv, mq3, mdo3, mqd, mdd, a, n_kv);
   return cudaGetLastError();
 }
@@ -980,7 +994,7 @@ static cudaError_t launch_dq_d(const BwdLaunch& L, cudaStream_t stream) {
   cudaError_t e =
       cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  bwd_dq_kernel<D><<<L.num_sms, kBwdThreads, smem, stream>>>(mk, mv, mq, mdo, a);
+  bwd_dq_kernel<D><<<L.num_sms, kKvThreads, smem, stream>>>(mk, mv, mq, mdo, a);
   return cudaGetLastError();
 }
 
