@@ -24,8 +24,9 @@
 //                      P^T  = exp2(S^T scale log2e - LSE2), dS^T = P^T (dP^T - D), written back
 //                             over S^T and dP^T in tensor memory as bf16
 //                      dV  += P^T dO,  dK += dS^T Q   (A from tensor memory, B MN-major)
-//   bwd_dq_kernel    query-stationary: one item per 128 query rows of one (g, b) routing list, or
-//                    of one head inside its own block (causal), walks the 128-key sub-tiles of b:
+//   bwd_dq_kernel    query-stationary: one item per 128 query rows of one (g, b) routing list (a
+//                    run of the densified rows) or of one head inside its own block (causal),
+//                    loaded as TMA tiles, walks the 128-key sub-tiles of b:
 //                      S = Q K_j^T, dP = dO V_j^T, dS = P (dP - D) over dP in tensor memory,
 //                      dQ += dS K_j
 //                    and adds scale * dQ once per item into the fp32 accumulator (red.global.add;
@@ -604,8 +605,10 @@ template <int D>
 __global__ void __launch_bounds__(kKvThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v,
-                  const __grid_constant__ CUtensorMap map_q,
-                  const __grid_constant__ CUtensorMap map_do, const BwdArgs a) {
+                  const __grid_constant__ CUtensorMap map_q3,
+                  const __grid_constant__ CUtensorMap map_do3,
+                  const __grid_constant__ CUtensorMap map_qd,
+                  const __grid_constant__ CUtensorMap map_dd, const BwdArgs a) {
   using C = QCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   QBars* bars = reinterpret_cast<QBars*>(smem + C::OFF_BARS);
@@ -637,8 +640,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&map_k);
     prefetch_tensormap(&map_v);
-    prefetch_tensormap(&map_q);
-    prefetch_tensormap(&map_do);
+    prefetch_tensormap(&map_q3);
+    prefetch_tensormap(&map_do3);
+    prefetch_tensormap(&map_qd);
+    prefetch_tensormap(&map_dd);
   }
   tc_fence_before();
   __syncthreads();
@@ -663,22 +668,22 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       if (it.kind == 0) continue;
       ok = wait_all(&bars->q_empty, (li & 1) ^ 1);
       if (!ok) break;
-      int rows4[4];
+      // the item's 128 query / dO rows as one TMA tile each: a run of the chunk's densified
+      // routed rows, or 128 consecutive tokens of one head (rows past the item are never used)
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int m = 4 * lane + e;
-        const int mm = m < it.rows ? m : 0;  // padding rows repeat row 0 (never written)
-        rows4[e] = it.kind == 1 ? a.T0 * a.H + __ldg(a.entries + it.start + mm) / a.topk
-                                : (it.start + mm) * a.H + it.h;
-      }
-      if (lane == 0) mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE);
-      __syncwarp();
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        tma_gather4(smem + C::OFF_Q + lane * 512 + c * 16384, &map_q, &bars->q_full, c * 64,
-                    rows4[0], rows4[1], rows4[2], rows4[3]);
-        tma_gather4(smem + C::OFF_DO + lane * 512 + c * 16384, &map_do, &bars->q_full, c * 64,
-                    rows4[0], rows4[1], rows4[2], rows4[3]);
+        for (int c = 0; c < D / 64; ++c) {
+          if (it.kind == 1) {
+            tma_load_2d(smem + C::OFF_Q + c * 16384, &map_qd, &bars->q_full, c * 64, it.start);
+            tma_load_2d(smem + C::OFF_DO + c * 16384, &map_dd, &bars->q_full, c * 64, it.start);
+          } else {
+            tma_load_3d(smem + C::OFF_Q + c * 16384, &map_q3, &bars->q_full, c * 64, it.h,
+                        it.start);
+            tma_load_3d(smem + C::OFF_DO + c * 16384, &map_do3, &bars->q_full, c * 64, it.h,
+                        it.start);
+          }
+        }
       }
       __syncwarp();
       ++li;
@@ -783,19 +788,21 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       if (it.kind == 0) continue;
       const bool rvalid = m < it.rows;
       int row = 0, t = 0;
+      float lse2 = INFINITY, dsv = 0.f;  // padding rows: p = 0
       if (rvalid) {
         if (it.kind == 1) {
+          // the densified row's columns (entry order = dense order)
           row = a.T0 * a.H + __ldg(a.entries + it.start + m) / a.topk;
-          t = row / a.H;
+          t = __ldg(a.col_t + it.start + m);
+          lse2 = __ldg(a.col_lse + it.start + m);
+          dsv = __ldg(a.col_d + it.start + m);
         } else {
           t = it.start + m;
           row = t * a.H + it.h;
+          lse2 = __ldg(a.lse + static_cast<size_t>(it.h) * a.T + t) * 1.4426950408889634f;
+          dsv = __ldg(a.dsum + row);
         }
       }
-      const float lse2 = rvalid ? __ldg(a.lse + static_cast<size_t>(row % a.H) * a.T + t) *
-                                      1.4426950408889634f
-                                : INFINITY;
-      const float dsv = rvalid ? __ldg(a.dsum + row) : 0.f;
       for (int j = 0; j < it.nsub; ++j, ++cs) {
         ok = wait_all(&bars->s_full, cs & 1);
         if (!ok) break;
@@ -984,17 +991,18 @@ static cudaError_t launch_dkdv_d(const BwdLaunch& L, cudaStream_t stream) {
 
 template <int D>
 static cudaError_t launch_dq_d(const BwdLaunch& L, cudaStream_t stream) {
-  CUtensorMap mk, mv, mq, mdo;
+  CUtensorMap mk, mv, mq3, mdo3, mqd, mdd;
   if (!make_kv_map(&mk, L.k, L.T, L.G, D) || !make_kv_map(&mv, L.v, L.T, L.G, D) ||
-      !make_q_rows_map(&mq, L.q, static_cast<long long>(L.T) * L.H, D) ||
-      !make_q_rows_map(&mdo, L.dout, static_cast<long long>(L.T) * L.H, D))
+      !make_kv_map(&mq3, L.q, L.T, L.H, D) || !make_kv_map(&mdo3, L.dout, L.T, L.H, D) ||
+      !make_rows_tile_map(&mqd, L.qd, std::max(L.dense_rows, 1LL), D) ||
+      !make_rows_tile_map(&mdd, L.dd, std::max(L.dense_rows, 1LL), D))
     return cudaErrorInvalidValue;
   const BwdArgs a = bwd_args(L);
   const int smem = std::max(QCfg<D>::SMEM, kOneCtaPerSmBytes);
   cudaError_t e =
       cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  bwd_dq_kernel<D><<<L.num_sms, kKvThreads, smem, stream>>>(mk, mv, mq, mdo, a);
+  bwd_dq_kernel<D><<<L.num_sms, kKvThreads, smem, stream>>>(mk, mv, mq3, mdo3, mqd, mdd, a);
   return cudaGetLastError();
 }
 
