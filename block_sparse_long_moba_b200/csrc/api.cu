@@ -396,19 +396,25 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu
     MOBA_LAUNCH(kRouteCount, s,
                 launch_route_count(idx, tb, P.T, Hq, Hkv, topk, P.NB, c.b0, c.nblk, c.T0, P.max_nb,
                                    counts, status, s));
-    MOBA_LAUNCH(kRouteScan, s, launch_route_scan(counts, NBK, cursor, tiles, n_tiles, s));
+    MOBA_LAUNCH(kRouteScan, s,
+                launch_route_scan(counts, NBK, cursor, tiles, n_tiles,
+                                  static_cast<long long>(P.max_tiles), status, s));
     MOBA_LAUNCH(kRouteScatter, s,
                 launch_route_scatter(idx, tb, P.T, Hq, Hkv, topk, P.NB, c.b0, c.nblk, c.T0,
-                                     P.max_nb, cursor, entries, s));
+                                     P.max_nb, cursor, entries,
+                                     static_cast<long long>(std::max<size_t>(P.max_entries, 1)),
+                                     status, s));
     if (qdense)
       MOBA_LAUNCH(kDensify, s,
                   launch_densify(entries, n_tiles + 1, q, Hq, topk, c.T0,
-                                 static_cast<long long>(P.max_entries), qdense, sms, s));
+                                 static_cast<long long>(P.max_entries), qdense, sms,
+                                 static_cast<long long>(P.T) * Hq, status, s));
     AttnLaunch A;
     A.q = q; A.k = k; A.v = v;
     A.tiles = tiles; A.n_routed = n_tiles; A.entries = entries; A.tb = tb;
     A.qdense = qdense;
     A.qdense_rows = static_cast<long long>(std::max<size_t>(P.max_entries, 1));
+    A.rows_cap = static_cast<long long>(P.max_rows);
     A.part_o = part_o; A.part_lse = part_lse; A.status = status;
     A.T = P.T; A.H = Hq; A.G = Hkv; A.d = d; A.B = block_size; A.topk = topk; A.NB = P.NB;
     A.b0 = c.b0; A.nblk = c.nblk; A.T0 = c.T0; A.scale = scale;
@@ -433,6 +439,7 @@ int read_status_word(const void* word_dev, void* stream) {
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOBA_ERR_CUDA;
   if (word == 0) return MOBA_OK;
   if (word == kDevTimeoutAttn || word == kDevDrainTimeout) return MOBA_ERR_TIMEOUT;
+  // kDevBadRouting, kDevSmemAlign, kDevCheckFail
   return MOBA_ERR_DEVICE_CHECK;
 }
 
@@ -733,10 +740,13 @@ int moba_attn_bwd(const void* q, const void* k, const void* v, const void* o, co
     MOBA_LAUNCH(kRouteCount, s,
                 launch_route_count(block_idx, tb, P.T, Hq, Hkv, topk, P.NB, c.b0, c.nblk, c.T0,
                                    P.max_nb, counts, status, s));
-    MOBA_LAUNCH(kRouteScan, s, launch_route_scan(counts, NBK, cursor, tiles, n_tiles, s));
+    MOBA_LAUNCH(kRouteScan, s,
+                launch_route_scan(counts, NBK, cursor, tiles, n_tiles,
+                                  static_cast<long long>(BP.max_entries / kItemRows + NBK + 1),
+                                  status, s));
     MOBA_LAUNCH(kRouteScatter, s,
                 launch_route_scatter(block_idx, tb, P.T, Hq, Hkv, topk, P.NB, c.b0, c.nblk, c.T0,
-                                     P.max_nb, cursor, entries, s));
+                                     P.max_nb, cursor, entries, B.dense_rows, status, s));
     MOBA_LAUNCH(kBwdAux, s, launch_bwd_densify(B, s));
     MOBA_LAUNCH(kBwdDkdv, s, launch_bwd_dkdv(B, s));
     MOBA_LAUNCH(kBwdDq, s, launch_bwd_dq(B, s));

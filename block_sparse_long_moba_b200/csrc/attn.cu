@@ -70,6 +70,7 @@ struct AttnArgs {
   float scale_log2;        // scale * log2(e)
   unsigned long long wait_ns;  // limit of one pipeline wait (abort drains use kDrainTimeoutNs)
   int diag_stall;              // diagnostics: the MMA issuer first waits on a barrier nobody arrives on
+  long long ent_cap, rows_cap, q_rows;  // sizes of entries, partial outputs, q rows (checks)
 };
 
 struct __align__(16) Item {
@@ -93,6 +94,9 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, int w, int n_rout
   it.slot = 0;
   if (w < n_routed) {
     const int4 tl = a.tiles[w];
+    if (!in_range(tl.x, static_cast<long long>(a.G) * a.NB, a.status) ||
+        !in_range(static_cast<long long>(tl.y) + tl.z - 1, a.ent_cap, a.status))
+      return it;  // (MOBA_CHECKS) a corrupt work item is skipped by every role alike
     it.kind = 1;
     it.g = tl.x / a.NB;
     it.b = tl.x % a.NB;
@@ -558,12 +562,13 @@ __global__ void __launch_bounds__(384, 1)
       for (int i = 0; i < 8; ++i) {
         const int r = 4 * i + (lane >> 3);
         const int pr = __shfl_sync(0xffffffffu, prev_prow, r);
-        if (pr >= 0)
+        if (pr >= 0 && in_range(pr, a.rows_cap, a.status))
           st_part(reinterpret_cast<uint4*>(a.part_o + static_cast<size_t>(pr) * D) + c,
                   *reinterpret_cast<const uint4*>(ep + r * 128 + ((c ^ (r & 7)) * 16)));
       }
       __syncwarp();
-      if (prev_prow >= 0) a.part_lse[prev_prow] = bars->ep_lse[q];
+      if (prev_prow >= 0 && in_range(prev_prow, a.rows_cap, a.status))
+        a.part_lse[prev_prow] = bars->ep_lse[q];
       return true;
     };
     for (uint32_t lt = 0;; ++lt) {
@@ -995,9 +1000,10 @@ __global__ void __launch_bounds__(384, 1)
             const int vb = __shfl_sync(0xffffffffu, qr4[2 * (i & 1) + 1], i >> 1);
             const int qr = r0 ? vb : va;
             const int m = 2 * i + r0;
-            const __nv_bfloat16* src = (qr >= 0) ? a.q + static_cast<size_t>(qr) * D + c * 8 : a.q;
+            const bool take = qr >= 0 && in_range(qr, a.q_rows, a.status);
+            const __nv_bfloat16* src = take ? a.q + static_cast<size_t>(qr) * D + c * 8 : a.q;
             cp_async_16(dst0 + (c >> 3) * 16384 + sw128_offset(m, (c & 7) * 8), src,
-                        qr >= 0 ? 16u : 0u);
+                        take ? 16u : 0u);
           }
           cp_async_wait_all();
           fence_proxy_async_smem();
@@ -1190,10 +1196,12 @@ __global__ void __launch_bounds__(384, 1)
           const int rr = 2 * i + (lane >> 4);
           const int pr = __shfl_sync(0xffffffffu, my_prow, rr);
           const uint4 v = *reinterpret_cast<const uint4*>(sP + p_offset(wrow0 + rr, c * 8));
-          if (pr >= 0) st_part(reinterpret_cast<uint4*>(a.part_o + static_cast<size_t>(pr) * D) + c, v);
+          if (pr >= 0 && in_range(pr, a.rows_cap, a.status))
+            st_part(reinterpret_cast<uint4*>(a.part_o + static_cast<size_t>(pr) * D) + c, v);
         }
       }
-      if (valid) a.part_lse[prow] = (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
+      if (valid && in_range(prow, a.rows_cap, a.status))
+        a.part_lse[prow] = (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
       // the P tile rows of this half are rewritten only by this warpgroup, after this point
       tc_fence_before();
     }
@@ -1295,6 +1303,9 @@ cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream) {
   a.scale_log2 = L.scale * 1.4426950408889634f;
   a.wait_ns = L.wait_ns > 0 ? L.wait_ns : kWaitTimeoutNs;
   a.diag_stall = L.diag_stall;
+  a.ent_cap = L.qdense_rows;
+  a.rows_cap = L.rows_cap;
+  a.q_rows = static_cast<long long>(L.T) * L.H;
   const int grid = L.grid > 0 ? L.grid : 1;
   // setmaxnreg.inc would wait forever if the launch had fewer registers than the split assumes
   {

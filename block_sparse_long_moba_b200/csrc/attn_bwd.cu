@@ -67,6 +67,7 @@ struct BwdArgs {
   int* status;
   int T, H, G, r, topk, NB, SPB;
   int T0, b0, nblk;         // the chunk: first token, first query block, query blocks
+  long long dense_rows;     // capacity of the chunk's entries and densified arrays (checks)
   float scale_log2, scale;
   unsigned long long wait_ns;
 };
@@ -134,14 +135,16 @@ __global__ void __launch_bounds__(256) bwd_densify_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ dout,
     const float* __restrict__ lse, const float* __restrict__ dsum, int T, int H, int topk, int T0,
     __nv_bfloat16* __restrict__ qd, __nv_bfloat16* __restrict__ dd, float* __restrict__ col_lse,
-    float* __restrict__ col_d, int* __restrict__ col_t) {
+    float* __restrict__ col_d, int* __restrict__ col_t, long long cap, int* __restrict__ status) {
   constexpr int LPR = D / 8;  // lanes per row
   const int n = *n_entries;
   const int sub = threadIdx.x % LPR;
   const long long stride = static_cast<long long>(gridDim.x) * (blockDim.x / LPR);
   for (long long p = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / LPR; p < n;
        p += stride) {
+    if (!in_range(p, cap, status)) break;
     const long long row = static_cast<long long>(T0) * H + __ldg(entries + p) / topk;
+    if (!in_range(row, static_cast<long long>(T) * H, status)) continue;
     const uint4 a = __ldg(reinterpret_cast<const uint4*>(q + row * D) + sub);
     const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + sub);
     __stcs(reinterpret_cast<uint4*>(qd + p * D) + sub, a);
@@ -179,6 +182,10 @@ __device__ __forceinline__ KvItem kv_item(const BwdArgs& a, int w) {
   it.bend = bstart + blen;
   it.rstart = x > 0 ? a.bucket_end[x - 1] : 0;
   it.rcount = a.bucket_end[x] - it.rstart;
+  if (it.rcount > 0 && (!in_range(it.rstart, a.dense_rows, a.status) ||
+                        !in_range(static_cast<long long>(it.rstart) + it.rcount - 1, a.dense_rows,
+                                  a.status)))
+    it.rcount = 0;  // (MOBA_CHECKS) a corrupt list is skipped by every role alike
   it.nrt = (it.rcount + 127) / 128;
   // the block's own rows belong to the chunk that holds the block
   const bool own = it.b >= a.b0 && it.b < a.b0 + a.nblk;
@@ -555,6 +562,9 @@ __device__ __forceinline__ QItem q_item(const BwdArgs& a, int w, int n_routed) {
     const int half = w & 1;
     it.rows = min(128, tl.z - half * 128);
     if (it.rows <= 0) return it;
+    if (!in_range(tl.x, static_cast<long long>(a.G) * a.NB, a.status) ||
+        !in_range(static_cast<long long>(tl.y) + tl.z - 1, a.dense_rows, a.status))
+      return it;  // (MOBA_CHECKS) a corrupt work item is skipped by every role alike
     it.kind = 1;
     it.g = tl.x / a.NB;
     it.b = tl.x % a.NB;
@@ -859,7 +869,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         tmem_wait_ld();
 #pragma unroll
         for (int x = 0; x < 32; ++x) reg_fence(qr[x]);
-        if (rvalid) {
+        if (rvalid && in_range(row, static_cast<long long>(a.T) * a.H, a.status)) {
 #pragma unroll
           for (int x = 0; x < 32; x += 4)
             red_add_v4(dst + c0 + x, __uint_as_float(qr[x]) * a.scale,
@@ -907,6 +917,7 @@ static BwdArgs bwd_args(const BwdLaunch& L) {
   a.T0 = L.T0;
   a.b0 = L.b0;
   a.nblk = L.nblk;
+  a.dense_rows = L.dense_rows;
   a.scale = L.scale;
   a.scale_log2 = L.scale * 1.4426950408889634f;
   a.wait_ns = L.wait_ns > 0 ? L.wait_ns : kWaitTimeoutNs;
@@ -960,11 +971,13 @@ cudaError_t launch_bwd_densify(const BwdLaunch& L, cudaStream_t stream) {
   if (L.d == 64)
     bwd_densify_kernel<64><<<grid, 256, 0, stream>>>(L.entries, L.n_routed + 1, q, dout, L.lse,
                                                      L.dsum, L.T, L.H, L.topk, L.T0, qd, dd,
-                                                     L.col_lse, L.col_d, L.col_t);
+                                                     L.col_lse, L.col_d, L.col_t, L.dense_rows,
+                                                     L.status);
   else
     bwd_densify_kernel<128><<<grid, 256, 0, stream>>>(L.entries, L.n_routed + 1, q, dout, L.lse,
                                                       L.dsum, L.T, L.H, L.topk, L.T0, qd, dd,
-                                                      L.col_lse, L.col_d, L.col_t);
+                                                      L.col_lse, L.col_d, L.col_t, L.dense_rows,
+                                                      L.status);
   return cudaGetLastError();
 }
 

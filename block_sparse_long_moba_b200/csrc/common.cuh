@@ -21,6 +21,25 @@ constexpr int kDevTimeoutAttn = 0x101;   // a pipeline wait ran out          -> 
 constexpr int kDevDrainTimeout = 0x102;  // an abort drain ran out            -> MOBA_ERR_TIMEOUT
 constexpr int kDevBadRouting = 0x201;    // a routing row breaks its contract -> MOBA_ERR_DEVICE_CHECK
 constexpr int kDevSmemAlign = 0x301;     // dynamic shared memory misaligned  -> MOBA_ERR_DEVICE_CHECK
+constexpr int kDevCheckFail = 0x401;     // an index check of the MOBA_CHECKS build failed
+                                         //                                   -> MOBA_ERR_DEVICE_CHECK
+
+// MOBA_CHECKS build (compiled with -DMOBA_CHECKS=1): every index the kernels derive from data on
+// the device (routing lists, work items, partial-row indices, densified rows) is checked against
+// the size of the buffer it indexes before use; a failing check records kDevCheckFail and the
+// access is skipped. In the normal build the checks compile to nothing.
+#ifndef MOBA_CHECKS
+#define MOBA_CHECKS 0
+#endif
+__device__ __forceinline__ bool in_range(long long x, long long n, int* status) {
+#if MOBA_CHECKS
+  if (x < 0 || x >= n) {
+    if (status) atomicCAS(status, 0, kDevCheckFail);
+    return false;
+  }
+#endif
+  return true;
+}
 
 // Block tables built on the device from cu_seqlens (workspace resident).
 struct BlockTables {

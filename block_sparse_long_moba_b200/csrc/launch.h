@@ -59,16 +59,17 @@ cudaError_t launch_route_count(const int32_t* idx, const BlockTables& tb, int T,
                                int* counts, int* status, cudaStream_t stream);
 
 cudaError_t launch_route_scan(int* counts, int nbk, int* cursor, int4* tiles, int* n_tiles,
-                              cudaStream_t stream);
+                              long long tiles_cap, int* status, cudaStream_t stream);
 
 cudaError_t launch_route_scatter(const int32_t* idx, const BlockTables& tb, int T, int H, int G,
                                  int topk, int NB, int b0, int nblk, int T0, int max_nb,
-                                 int* cursor, int* entries, cudaStream_t stream);
+                                 int* cursor, int* entries, long long ent_cap, int* status,
+                                 cudaStream_t stream);
 
 // d = 64: copies the query row of every routed entry of the chunk into qdense (row = entry).
 cudaError_t launch_densify(const int* entries, const int* n_entries, const void* q, int H,
                            int topk, int T0, long long max_entries, void* qdense, int num_sms,
-                           cudaStream_t stream);
+                           long long q_rows, int* status, cudaStream_t stream);
 
 struct AttnLaunch {
   const void* q;
@@ -78,7 +79,8 @@ struct AttnLaunch {
   const int* n_routed;
   const int* entries;
   const void* qdense;      // d = 64: routed query rows, one per entry (nullptr otherwise)
-  long long qdense_rows;   // rows of qdense
+  long long qdense_rows;   // rows of qdense (= capacity of the entries list)
+  long long rows_cap;      // partial-output rows
   BlockTables tb;
   void* part_o;
   float* part_lse;

@@ -91,7 +91,7 @@ template <bool kScatter>
 __global__ void __launch_bounds__(256) route_pass_kernel(
     const int32_t* __restrict__ idx, BlockTables tb, int T, int H, int G, int topk, int NB,
     int b0, int T0, int* __restrict__ counts, int* __restrict__ cursor,
-    int* __restrict__ entries, int* __restrict__ status) {
+    int* __restrict__ entries, int* __restrict__ status, long long ent_cap) {
   extern __shared__ int hist[];
   const int b = b0 + blockIdx.x, g = blockIdx.y;
   const int s = tb.blk_seq[b];
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(256) route_pass_kernel(
       const int j = __ldg(rp + slot);
       if (j >= 0 && j < i) {
         const int pos = atomicAdd(&hist[j], 1);
-        entries[pos] = prow + slot;
+        if (in_range(pos, ent_cap, status)) entries[pos] = prow + slot;
       }
     }
   }
@@ -155,7 +155,9 @@ __global__ void __launch_bounds__(256) route_pass_kernel(
 __global__ void __launch_bounds__(1024) route_scan_kernel(int* __restrict__ counts, int nbk,
                                                           int* __restrict__ cursor,
                                                           int4* __restrict__ tiles,
-                                                          int* __restrict__ n_tiles) {
+                                                          int* __restrict__ n_tiles,
+                                                          long long tiles_cap,
+                                                          int* __restrict__ status) {
   __shared__ int ws_c[32], ws_t[32];
   const int tid = threadIdx.x, nt = blockDim.x;
   const int per = (nbk + nt - 1) / nt;
@@ -205,7 +207,8 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int* __restrict__ coun
     const int c = counts[x];
     cursor[x] = off;
     for (int y = 0; y * kItemRows < c; ++y)
-      tiles[toff + y] = make_int4(x, off + y * kItemRows, min(kItemRows, c - y * kItemRows), 0);
+      if (in_range(toff + y, tiles_cap, status))
+        tiles[toff + y] = make_int4(x, off + y * kItemRows, min(kItemRows, c - y * kItemRows), 0);
     toff += (c + kItemRows - 1) / kItemRows;
     off += c;
     counts[x] = 0;
@@ -224,14 +227,18 @@ __global__ void __launch_bounds__(256) densify_kernel(const int* __restrict__ en
                                                       const int* __restrict__ n_entries,
                                                       const __nv_bfloat16* __restrict__ q, int H,
                                                       int topk, int T0,
-                                                      __nv_bfloat16* __restrict__ qdense) {
+                                                      __nv_bfloat16* __restrict__ qdense,
+                                                      long long cap, long long q_rows,
+                                                      int* __restrict__ status) {
   const int n = *n_entries;
   const int lane8 = threadIdx.x & 7;
   const long long stride = static_cast<long long>(gridDim.x) * (blockDim.x >> 3);
   for (long long p = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 3; p < n;
        p += stride) {
+    if (!in_range(p, cap, status)) break;
     const int e = __ldg(entries + p);
     const long long row = static_cast<long long>(T0) * H + e / topk;  // t * H + h
+    if (!in_range(row, q_rows, status)) continue;
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(q + row * 64) + lane8);
     __stcs(reinterpret_cast<uint4*>(qdense + p * 64) + lane8, v);
   }
@@ -251,36 +258,39 @@ cudaError_t launch_route_count(const int32_t* idx, const BlockTables& tb, int T,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   route_pass_kernel<false><<<dim3(nblk, G), 256, smem, stream>>>(
-      idx, tb, T, H, G, topk, NB, b0, T0, counts, nullptr, nullptr, status);
+      idx, tb, T, H, G, topk, NB, b0, T0, counts, nullptr, nullptr, status, 0);
   return cudaGetLastError();
 }
 
 cudaError_t launch_route_scan(int* counts, int nbk, int* cursor, int4* tiles, int* n_tiles,
-                              cudaStream_t stream) {
-  route_scan_kernel<<<1, 1024, 0, stream>>>(counts, nbk, cursor, tiles, n_tiles);
+                              long long tiles_cap, int* status, cudaStream_t stream) {
+  route_scan_kernel<<<1, 1024, 0, stream>>>(counts, nbk, cursor, tiles, n_tiles, tiles_cap,
+                                            status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_densify(const int* entries, const int* n_entries, const void* q, int H,
                            int topk, int T0, long long max_entries, void* qdense, int num_sms,
-                           cudaStream_t stream) {
+                           long long q_rows, int* status, cudaStream_t stream) {
   const long long want = (max_entries + 31) / 32;  // 32 rows per CTA pass
   const int grid = static_cast<int>(std::min<long long>(std::max(want, 1LL), 8LL * num_sms));
   densify_kernel<<<grid, 256, 0, stream>>>(entries, n_entries,
                                            static_cast<const __nv_bfloat16*>(q), H, topk, T0,
-                                           static_cast<__nv_bfloat16*>(qdense));
+                                           static_cast<__nv_bfloat16*>(qdense), max_entries,
+                                           q_rows, status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_route_scatter(const int32_t* idx, const BlockTables& tb, int T, int H, int G,
                                  int topk, int NB, int b0, int nblk, int T0, int max_nb,
-                                 int* cursor, int* entries, cudaStream_t stream) {
+                                 int* cursor, int* entries, long long ent_cap, int* status,
+                                 cudaStream_t stream) {
   const int smem = max_nb * 4;
   cudaError_t e = cudaFuncSetAttribute(route_pass_kernel<true>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   route_pass_kernel<true><<<dim3(nblk, G), 256, smem, stream>>>(
-      idx, tb, T, H, G, topk, NB, b0, T0, nullptr, cursor, entries, nullptr);
+      idx, tb, T, H, G, topk, NB, b0, T0, nullptr, cursor, entries, status, ent_cap);
   return cudaGetLastError();
 }
 

@@ -13,7 +13,9 @@ from typing import Optional, Sequence, Tuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmoba.so")
+# MOBA_CHECKS=1 in the environment selects the build with device-side index checks
+LIB_PATH = os.path.join(_HERE, "libmoba_checks.so" if os.environ.get("MOBA_CHECKS") == "1"
+                        else "libmoba.so")
 
 STATUS = {0: "MOBA_OK", -1: "MOBA_ERR_ARG", -2: "MOBA_ERR_UNSUPPORTED", -3: "MOBA_ERR_WORKSPACE",
           -4: "MOBA_ERR_CUDA", -5: "MOBA_ERR_DEVICE_CHECK", -6: "MOBA_ERR_TIMEOUT"}
@@ -42,7 +44,8 @@ _lib = None
 
 
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Load libmoba.so (build it with `python -m block_sparse_long_moba_b200.build`)."""
+    """Load libmoba.so, or libmoba_checks.so when MOBA_CHECKS=1 (build them with
+    `python -m block_sparse_long_moba_b200.build [--checks]`)."""
     global _lib
     if _lib is not None:
         return _lib
