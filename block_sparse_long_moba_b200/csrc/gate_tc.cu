@@ -45,7 +45,7 @@ struct GateCfg {
   static constexpr int M = (KCAP <= 16) ? 32 : 64;           // groups of pass 1
   static constexpr int CB = (KCAP <= 16) ? 32 : 64;          // candidate slots per row
   static constexpr int Q_BYTES = kTile * D * 2;             // one 128-row query tile
-  static constexpr int CAND_BYTES = 2 * CB * 128 * 8;        // [2][CB][128] fp32 + [2][CB][128] int
+  static constexpr int CAND_BYTES = 2 * CB * 128 * 8;        // [2][CB][128] (fp32 score, int block)
   // centroid rows resident at once (a multiple of 16): what is left of the CTA's shared memory
   static constexpr int CAP = (D == 128) ? (KCAP <= 16 ? 192 : 64) : (KCAP <= 16 ? 512 : 256);
   static constexpr int B_BYTES = 2 * NCB * CAP * 128;        // hi + lo, 128 B per row per block
@@ -152,6 +152,7 @@ __global__ void __launch_bounds__(256, 1)
                    const uint8_t* __restrict__ split, int nb_pad) {
   using C = GateCfg<D, KCAP>;
   constexpr int M = C::M, CB = C::CB;
+  constexpr int STEP = (M == 32) ? 64 : 32;
   extern __shared__ __align__(1024) uint8_t smem[];
   GateBars* bars = reinterpret_cast<GateBars*>(smem + C::OFF_BARS);
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -182,15 +183,26 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t tmem = bars->tmem_base;
   const uint32_t t_s = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + wg * 2 * C::PIECE;
   uint8_t* sQ = smem + wg * C::Q_BYTES;
-  // this warpgroup's candidate buffer [CB][128] scores + [CB][128] blocks (pass 2), the scores
-  // part reused as staging [32][128] (pass 3)
-  float* cand = reinterpret_cast<float*>(smem + C::OFF_STAGE) + wg * CB * 128;
-  int* candi = reinterpret_cast<int*>(smem + C::OFF_STAGE) + 2 * CB * 128 + wg * CB * 128;
+  // this warpgroup's candidate buffer [CB][128] of (score bits, block) pairs (pass 2), the score
+  // words reused as staging [32][128] (pass 3), the block words as the selected list's staging
+  uint2* cand = reinterpret_cast<uint2*>(smem + C::OFF_STAGE) + wg * CB * 128;
+  const uint32_t cand_base = smem_u32(cand + row);  // this row's slot 0 (slots 1024 bytes apart)
+  // predicated append, no branch: if s >= t, store (s, j) in the slot at address a, advance a
+  auto append_if_ge = [](uint32_t& a, float sv, float t, int j) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ge.f32 p, %1, %2;\n @p st.shared.v2.b32 [%0], {%1, %3};\n"
+        " @p add.u32 %0, %0, 1024;\n}\n"
+        : "+r"(a)
+        : "f"(sv), "f"(t), "r"(j)
+        : "memory");
+  };
   uint32_t chunk_phase = 0;   // chunk_full phase (pre-split centroids)
   bool chunk_pending = false; // a chunk copy issued by thread 0 that no wait has seen land
   const uint32_t sBa = smem_u32(smem + C::OFF_B);
   const int r = H / G;
   const int ksel = topk - 1;
+  // rows of the routing are written as 16-byte pieces when each row starts on a 16-byte boundary
+  const bool vec_out = (topk & 3) == 0 && (reinterpret_cast<uintptr_t>(idx) & 15) == 0;
   const uint64_t TO = kWaitTimeoutNs;
   uint32_t qphase = 0;  // q_full phase of this warpgroup
   uint32_t npiece = 0;  // score pieces issued by this warpgroup (TMEM buffer npiece & 1)
@@ -284,14 +296,15 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
       for (int x = 0; x < M; ++x) gmax[x] = -INFINITY;
       float tau = -INFINITY, tau_star = INFINITY;
-      int cnt = 0, tie_budget = 0, pos = 0;
+      int cnt = 0, tie_budget = 0;
+      unsigned long long sel_mask = 0;  // selected candidate slots (ksel bits)
       bool overflow = false;
-      TopList<KCAP> top;
-      top.init(ksel);
+      TopList<KCAP> top;  // the third pass's running list (initialised there)
       bool q_ready = false;
       for (int pass = 0; pass < 3; ++pass) {
         // the third pass only runs for rows whose candidates overflowed (CTA-uniform decision)
         if (pass == 2 && !__syncthreads_or(overflow && scored && row < rows)) break;
+        if (pass == 2) top.init(ksel);
         for (int ch = 0; ch < nchunks; ++ch) {
           const int c0 = ch * C::CAP;
           const int n = min(C::CAP, i_max - c0);
@@ -415,60 +428,100 @@ __global__ void __launch_bounds__(256, 1)
             if (__all_sync(0xffffffffu, w)) {
               tc_fence_after();
               const uint32_t tb = t_s + (pc & 1) * C::PIECE;
-              for (int cc = 0; cc < np; cc += 32) {
-                uint32_t sr[32];
-                tmem_ld32(tb + cc, sr);
+              // STEP columns per TMEM wait (64 with 32 groups, where both halves feed the same
+              // group maxima; 32 with 64 groups, for registers); columns past the tile's last past
+              // block read as -inf, so the per-score work below needs no bounds test
+              for (int cc = 0; cc < np; cc += STEP) {
+                uint32_t sa[32], sb[32];
+                const bool two = STEP == 64 && cc + 32 < np;  // warpgroup-uniform
+                tmem_ld32(tb + cc, sa);
+                if (two) tmem_ld32(tb + cc + 32, sb);
                 tmem_wait_ld();
 #pragma unroll
-                for (int x = 0; x < 32; ++x) reg_fence(sr[x]);
-                const int jb = c0 + p0 + cc;  // block of column x is jb + x (jb % 32 == 0)
+                for (int x = 0; x < 32; ++x) {
+                  reg_fence(sa[x]);
+                  if (STEP == 64) reg_fence(sb[x]);
+                }
+                const int lim = np - cc;  // valid columns of the 64: c < lim
+                if (lim < STEP) {
+#pragma unroll
+                  for (int x = 0; x < 32; ++x) {
+                    if (x >= lim) sa[x] = __float_as_uint(-INFINITY);
+                    if (STEP == 64 && 32 + x >= lim) sb[x] = __float_as_uint(-INFINITY);
+                  }
+                }
+                const int jb = c0 + p0 + cc;  // block of sa[x] is jb + x, of sb[x] jb + 32 + x
                 if (pass == 0) {
                   // group maxima, column j in group j mod M
-                  if (M == 32 || (jb & 32) == 0) {
+                  if (M == 32) {
 #pragma unroll
                     for (int x = 0; x < 32; ++x)
-                      if (cc + x < np) gmax[x] = fmaxf(gmax[x], __uint_as_float(sr[x]));
+                      gmax[x] = fmax3(gmax[x], __uint_as_float(sa[x]), __uint_as_float(sb[x]));
+                  } else if ((jb & 32) == 0) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) gmax[x] = fmaxf(gmax[x], __uint_as_float(sa[x]));
                   } else {
 #pragma unroll
                     for (int x = 0; x < 32; ++x)
-                      if (cc + x < np)
-                        gmax[(32 + x) % M] = fmaxf(gmax[(32 + x) % M], __uint_as_float(sr[x]));
+                      gmax[(32 + x) % M] = fmaxf(gmax[(32 + x) % M], __uint_as_float(sa[x]));
                   }
                 } else if (pass == 1) {
-                  // every score >= tau is a candidate, kept with its block (ascending)
+                  // every score >= tau is a candidate, kept with its block (ascending). While at
+                  // least eight slots are free, eight columns at a time append without a capacity
+                  // test ((score, block) pairs to cand[slot][row]).
+                  auto append = [&](const uint32_t (&v)[32], int jb0) {
 #pragma unroll
-                  for (int x = 0; x < 32; ++x) {
-                    const float sv = __uint_as_float(sr[x]);
-                    if (cc + x < np && sv >= tau) {
-                      if (cnt < CB) {
-                        cand[cnt * 128 + row] = sv;
-                        candi[cnt * 128 + row] = jb + x;
+                    for (int x0 = 0; x0 < 32; x0 += 8) {
+                      if (cnt <= CB - 8) {
+                        uint32_t cp = cand_base + static_cast<uint32_t>(cnt) * 1024u;
+#pragma unroll
+                        for (int x = x0; x < x0 + 8; ++x)
+                          append_if_ge(cp, __uint_as_float(v[x]), tau, jb0 + x);
+                        cnt = static_cast<int>((cp - cand_base) >> 10);
+                      } else {
+#pragma unroll
+                        for (int x = x0; x < x0 + 8; ++x) {
+                          const float sv = __uint_as_float(v[x]);
+                          if (sv >= tau) {
+                            if (cnt < CB) {
+                              cand[cnt * 128 + row] = make_uint2(__float_as_uint(sv), jb0 + x);
+                            }
+                            ++cnt;
+                          }
+                        }
                       }
-                      ++cnt;
                     }
-                  }
+                  };
+                  append(sa, jb);
+                  if (two) append(sb, jb + 32);
                 } else {
                   // rows whose candidates overflowed keep a running top list instead
-                  const float thr0 = top.thr();
-                  uint32_t mask = 0;
-                  if (overflow) {
 #pragma unroll
-                    for (int x = 0; x < 32; ++x)
-                      if (cc + x < np && __uint_as_float(sr[x]) > thr0) mask |= 1u << x;
-                  }
-                  if (__any_sync(0xffffffffu, mask != 0)) {
+                  for (int hh = 0; hh < 2; ++hh) {
+                    if (hh == 1 && !two) break;
+                    const uint32_t(&sr)[32] = hh ? sb : sa;
+                    const int jh = jb + 32 * hh;
+                    const float thr0 = top.thr();
+                    uint32_t mask = 0;
                     if (overflow) {
 #pragma unroll
-                      for (int x = 0; x < 32; ++x) cand[x * 128 + row] = __uint_as_float(sr[x]);
+                      for (int x = 0; x < 32; ++x)
+                        if (__uint_as_float(sr[x]) > thr0) mask |= 1u << x;
                     }
-                    while (__any_sync(0xffffffffu, mask != 0)) {
-                      if (mask) {
-                        const int x = __ffs(mask) - 1;
-                        mask &= mask - 1;
-                        top.offer(cand[x * 128 + row], jb + x);
+                    if (__any_sync(0xffffffffu, mask != 0)) {
+                      if (overflow) {
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) cand[x * 128 + row].x = sr[x];
                       }
+                      while (__any_sync(0xffffffffu, mask != 0)) {
+                        if (mask) {
+                          const int x = __ffs(mask) - 1;
+                          mask &= mask - 1;
+                          top.offer(__uint_as_float(cand[x * 128 + row].x), jh + x);
+                        }
+                      }
+                      __syncwarp();
                     }
-                    __syncwarp();
                   }
                 }
               }
@@ -486,21 +539,38 @@ __global__ void __launch_bounds__(256, 1)
         } else if (pass == 1) {
           overflow = cnt > CB;
           if (!overflow) {
+            // the exact ksel-th best score tau* among the candidates (a sort of 32 values when
+            // they fit, the buffer's CB otherwise), and how many of the selected tie with it
             float cv[CB];
 #pragma unroll
-            for (int x = 0; x < CB; ++x) cv[x] = (x < cnt) ? cand[x * 128 + row] : -INFINITY;
-            bitonic_desc_f<CB>(cv);
-            tau_star = kth_of_sorted<CB>(cv, ksel);
+            for (int x = 0; x < CB; ++x)
+              cv[x] = (x < cnt) ? __uint_as_float(cand[x * 128 + row].x) : -INFINITY;
             int above = 0;
+            if (CB > 32 && cnt <= 32) {
+              float c32[32];
 #pragma unroll
-            for (int x = 0; x < CB; ++x) above += (cv[x] > tau_star) ? 1 : 0;
+              for (int x = 0; x < 32; ++x) c32[x] = cv[x];
+              bitonic_desc_f<32>(c32);
+              tau_star = kth_of_sorted<32>(c32, ksel);
+#pragma unroll
+              for (int x = 0; x < 32; ++x) above += (c32[x] > tau_star) ? 1 : 0;
+            } else {
+              bitonic_desc_f<CB>(cv);
+              tau_star = kth_of_sorted<CB>(cv, ksel);
+#pragma unroll
+              for (int x = 0; x < CB; ++x) above += (cv[x] > tau_star) ? 1 : 0;
+            }
             tie_budget = ksel - above;
-            // the buffer is in ascending block order: blocks above tau*, then the lowest ties
-            for (int x = 0; x < cnt; ++x) {
-              const float sv = cand[x * 128 + row];
-              if (sv > tau_star || (sv == tau_star && tie_budget-- > 0)) {
-                if (row < rows) out[pos] = candi[x * 128 + row];
-                ++pos;
+            // the buffer is in ascending block order: the selection is the blocks above tau* and
+            // the lowest ties, marked in a bit mask (loads independent of the running tie count)
+            int ties = 0;
+#pragma unroll
+            for (int x = 0; x < CB; ++x) {
+              if (x < cnt) {
+                const float sv = __uint_as_float(cand[x * 128 + row].x);
+                const bool tie = sv == tau_star && ties < tie_budget;
+                ties += tie ? 1 : 0;
+                if (sv > tau_star || tie) sel_mask |= 1ull << x;
               }
             }
           }
@@ -512,7 +582,27 @@ __global__ void __launch_bounds__(256, 1)
         if (t < ntiles) load_q(t);
       }
       if (!scored || row >= rows || !ok) continue;
-      if (overflow) {
+      if (!overflow) {
+        // the ksel selected blocks (the set bits of sel_mask, ascending) and the current block,
+        // as 16-byte pieces of the row when its length and address allow
+        unsigned long long m = sel_mask;
+        auto sel = [&](int x) {
+          if (x >= ksel) return i_t;
+          const int slot = __ffsll(static_cast<long long>(m)) - 1;
+          m &= m - 1;
+          return static_cast<int>(cand[slot * 128 + row].y);
+        };
+        if (vec_out) {
+          for (int x = 0; x < topk; x += 4) {
+            const int a0 = sel(x), a1 = sel(x + 1), a2 = sel(x + 2), a3 = sel(x + 3);
+            *reinterpret_cast<int4*>(out + x) = make_int4(a0, a1, a2, a3);
+          }
+        } else {
+          for (int x = 0; x < topk; ++x) out[x] = sel(x);
+        }
+        continue;
+      }
+      {
         // the ksel real entries of the running list (sentinels map to INT_MAX), ascending
         int sel[KCAP];
 #pragma unroll
