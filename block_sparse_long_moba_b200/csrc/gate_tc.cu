@@ -52,15 +52,23 @@ struct GateCfg {
   static constexpr int OFF_B = 2 * Q_BYTES;                  // one Q buffer per warpgroup
   static constexpr int OFF_STAGE = OFF_B + B_BYTES;          // candidate buffer / staging
   static constexpr int OFF_BARS = OFF_STAGE + CAND_BYTES;
-  static constexpr int SMEM_BYTES = OFF_BARS + 256;
+  static constexpr int SMEM_BYTES = OFF_BARS + 384;
   static constexpr int PIECE = 128;                          // MMA N (scores per TMEM buffer)
+  // ring mode (past blocks beyond CAP): RS slots of PR centroid rows each, PR a multiple of 16
+  static constexpr int PR = CAP >= 256 ? 128 : CAP / 2;
+  static constexpr int RS = CAP / PR;
 };
+static_assert(GateCfg<64, 16>::RS <= 4 && GateCfg<64, 32>::RS <= 4 && GateCfg<128, 16>::RS <= 4 &&
+                  GateCfg<128, 32>::RS <= 4 && GateCfg<128, 16>::CAP % GateCfg<128, 16>::PR == 0 &&
+                  GateCfg<128, 16>::PR % 16 == 0 && GateCfg<128, 32>::PR % 16 == 0,
+              "ring slots");
 static_assert(GateCfg<128, 16>::SMEM_BYTES <= 232448 && GateCfg<64, 16>::SMEM_BYTES <= 232448 &&
                   GateCfg<128, 32>::SMEM_BYTES <= 232448 && GateCfg<64, 32>::SMEM_BYTES <= 232448,
               "shared memory budget of one CTA");
 
 struct GateBars {
   uint64_t q_full[2], mma_done[2][2], chunk_full;
+  uint64_t slot_full[4], slot_free[4];  // ring mode
   uint32_t tmem_base;
   int abort_flag;
   int red[32];
@@ -169,6 +177,10 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(&bars->mma_done[x][1], 1);
     }
     mbar_init(&bars->chunk_full, 1);
+    for (int x = 0; x < C::RS; ++x) {
+      mbar_init(&bars->slot_full[x], 1);
+      mbar_init(&bars->slot_free[x], 2);  // one arrival per warpgroup
+    }
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -197,6 +209,8 @@ __global__ void __launch_bounds__(256, 1)
         : "memory");
   };
   uint32_t chunk_phase = 0;   // chunk_full phase (pre-split centroids)
+  uint32_t ring_l = 0;        // ring loads so far (CTA-uniform count)
+  uint32_t ring_issued = 0;   // ring loads issued by thread 0
   bool chunk_pending = false; // a chunk copy issued by thread 0 that no wait has seen land
   const uint32_t sBa = smem_u32(smem + C::OFF_B);
   const int r = H / G;
@@ -257,6 +271,8 @@ __global__ void __launch_bounds__(256, 1)
     const int i_max = i_last > ksel && ksel > 0 ? i_last : 0;
     const int base = seq_block_base(cu, s, B, bars->red);
     const int nchunks = (i_max + C::CAP - 1) / C::CAP;
+    // past blocks beyond the resident capacity stream through a ring of slots (pre-split only)
+    const bool ring = split != nullptr && nchunks > 1;
     auto load_q = [&](int tile) {  // TMA of a query tile into this warpgroup's buffer
       int i_t, h_t, t0_t, rows_t;
       tile_info(tile, i_t, h_t, t0_t, rows_t);
@@ -284,6 +300,40 @@ __global__ void __launch_bounds__(256, 1)
       int i_t = 0, h = 0, t0 = 0, rows = 0;
       if (tile < ntiles) tile_info(tile, i_t, h, t0, rows);
       const bool scored = tile < ntiles && rows > 0 && i_t > ksel && ksel > 0;
+      // past blocks this warpgroup scores, and the pair's (both warpgroups') number of ring pieces
+      const int n_self = scored ? i_t : 0;
+      int n_pair = n_self;
+      {
+        const int other = 2 * p + 1 - wg;
+        int i_o = 0, h_o = 0, t0_o = 0, rows_o = 0;
+        if (other < ntiles) tile_info(other, i_o, h_o, t0_o, rows_o);
+        if (other < ntiles && rows_o > 0 && i_o > ksel && ksel > 0) n_pair = max(n_pair, i_o);
+      }
+      const int K_pair = (n_pair + C::PR - 1) / C::PR;
+      // (thread 0) ring load Lm: centroid rows of piece k into slot Lm % RS, once both warpgroups
+      // have released the slot's previous load. A wait that runs out raises the CTA's abort flag
+      // (every later wait then fails, and `ok` turns false at the next warpgroup barrier), so
+      // `ok` itself is left alone here: it must stay uniform inside the issuing warp.
+      auto ring_load = [&](uint32_t Lm, int k) {
+        if (!ok) return;
+        const uint32_t sl = Lm % C::RS;
+        if (Lm >= static_cast<uint32_t>(C::RS) &&
+            !mbar_wait_bounded(&bars->slot_free[sl], ((Lm / C::RS) - 1) & 1, abort_flag, status,
+                               kDevTimeoutAttn, TO))
+          return;
+        const int c0r = k * C::PR;
+        const int rows_pad = (min(C::PR, n_pair - c0r) + 15) & ~15;
+        mbar_arrive_expect_tx(&bars->slot_full[sl], 2 * C::NCB * rows_pad * 128);
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+          for (int at = 0; at < C::NCB; ++at)
+            bulk_load(smem + C::OFF_B + c_offset<D, KCAP>(part, static_cast<int>(sl) * C::PR, 64 * at),
+                      split + ((static_cast<size_t>(g * 2 + part) * C::NCB + at) * nb_pad + base +
+                               c0r) * 128,
+                      rows_pad * 128, &bars->slot_full[sl]);
+        ++ring_issued;
+      };
       int32_t* out = idx + (static_cast<size_t>(h) * T + t0 + row) * topk;
       if (tile < ntiles && rows > 0 && !scored && row < rows) {
         // few causal blocks or topk == 1: the selection is fixed, no scores needed
@@ -301,10 +351,198 @@ __global__ void __launch_bounds__(256, 1)
       bool overflow = false;
       TopList<KCAP> top;  // the third pass's running list (initialised there)
       bool q_ready = false;
+      // scores of 128 rows x np past blocks (from centroid rows row_off.. of the B region) into
+      // TMEM buffer `buf`; one converged warp of the warpgroup issues
+      const uint32_t qa = smem_u32(sQ);
+      auto issue_rows = [&](int row_off, int np, uint32_t buf) {
+        const int nmma = (np + 15) & ~15;
+        const uint32_t idesc = idesc_bf16_f32(128, nmma, 0, 0);
+        tc_fence_after();
+#pragma unroll
+        for (int sp = 0; sp < 2; ++sp) {
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t aoff = (ks >> 2) * 16384 + (ks & 3) * 32;
+            const uint32_t boff = static_cast<uint32_t>(sp * C::NCB * C::CAP * 128 +
+                                                        (ks >> 2) * C::CAP * 128 + row_off * 128 +
+                                                        (ks & 3) * 32);
+            mma_ss_elect(tmem + wg * 2 * C::PIECE + buf * C::PIECE,
+                         smem_desc_sw128(qa + aoff, 16, 1024),
+                         smem_desc_sw128(sBa + boff, 16, 1024), idesc, (sp > 0 || ks > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit_elect(&bars->mma_done[wg][buf]);
+      };
+      // the pass's work on one piece of scores (TMEM buffer of piece number pc; its columns are
+      // past blocks gb .. gb + np - 1)
+      auto select_piece = [&](int pass, uint32_t pc, int gb, int np) {
+          tc_fence_after();
+          const uint32_t tb = t_s + (pc & 1) * C::PIECE;
+          // STEP columns per TMEM wait (64 with 32 groups, where both halves feed the same
+          // group maxima; 32 with 64 groups, for registers); columns past the tile's last past
+          // block read as -inf, so the per-score work below needs no bounds test
+          for (int cc = 0; cc < np; cc += STEP) {
+            uint32_t sa[32], sb[32];
+            const bool two = STEP == 64 && cc + 32 < np;  // warpgroup-uniform
+            tmem_ld32(tb + cc, sa);
+            if (two) tmem_ld32(tb + cc + 32, sb);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+              reg_fence(sa[x]);
+              if (STEP == 64) reg_fence(sb[x]);
+            }
+            const int lim = np - cc;  // valid columns of the 64: c < lim
+            if (lim < STEP) {
+#pragma unroll
+              for (int x = 0; x < 32; ++x) {
+                if (x >= lim) sa[x] = __float_as_uint(-INFINITY);
+                if (STEP == 64 && 32 + x >= lim) sb[x] = __float_as_uint(-INFINITY);
+              }
+            }
+            const int jb = gb + cc;  // block of sa[x] is jb + x, of sb[x] jb + 32 + x
+            if (pass == 0) {
+              // group maxima, column j in group j mod M
+              if (M == 32) {
+#pragma unroll
+                for (int x = 0; x < 32; ++x)
+                  gmax[x] = fmax3(gmax[x], __uint_as_float(sa[x]), __uint_as_float(sb[x]));
+              } else if ((jb & 32) == 0) {
+#pragma unroll
+                for (int x = 0; x < 32; ++x) gmax[x] = fmaxf(gmax[x], __uint_as_float(sa[x]));
+              } else {
+#pragma unroll
+                for (int x = 0; x < 32; ++x)
+                  gmax[(32 + x) % M] = fmaxf(gmax[(32 + x) % M], __uint_as_float(sa[x]));
+              }
+            } else if (pass == 1) {
+              // every score >= tau is a candidate, kept with its block (ascending). While at
+              // least eight slots are free, eight columns at a time append without a capacity
+              // test ((score, block) pairs to cand[slot][row]).
+              auto append = [&](const uint32_t (&v)[32], int jb0) {
+#pragma unroll
+                for (int x0 = 0; x0 < 32; x0 += 8) {
+                  if (cnt <= CB - 8) {
+                    uint32_t cp = cand_base + static_cast<uint32_t>(cnt) * 1024u;
+#pragma unroll
+                    for (int x = x0; x < x0 + 8; ++x)
+                      append_if_ge(cp, __uint_as_float(v[x]), tau, jb0 + x);
+                    cnt = static_cast<int>((cp - cand_base) >> 10);
+                  } else {
+#pragma unroll
+                    for (int x = x0; x < x0 + 8; ++x) {
+                      const float sv = __uint_as_float(v[x]);
+                      if (sv >= tau) {
+                        if (cnt < CB) {
+                          cand[cnt * 128 + row] = make_uint2(__float_as_uint(sv), jb0 + x);
+                        }
+                        ++cnt;
+                      }
+                    }
+                  }
+                }
+              };
+              append(sa, jb);
+              if (two) append(sb, jb + 32);
+            } else {
+              // rows whose candidates overflowed keep a running top list instead
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                if (hh == 1 && !two) break;
+                const uint32_t(&sr)[32] = hh ? sb : sa;
+                const int jh = jb + 32 * hh;
+                const float thr0 = top.thr();
+                uint32_t mask = 0;
+                if (overflow) {
+#pragma unroll
+                  for (int x = 0; x < 32; ++x)
+                    if (__uint_as_float(sr[x]) > thr0) mask |= 1u << x;
+                }
+                if (__any_sync(0xffffffffu, mask != 0)) {
+                  if (overflow) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) cand[x * 128 + row].x = sr[x];
+                  }
+                  while (__any_sync(0xffffffffu, mask != 0)) {
+                    if (mask) {
+                      const int x = __ffs(mask) - 1;
+                      mask &= mask - 1;
+                      top.offer(__uint_as_float(cand[x * 128 + row].x), jh + x);
+                    }
+                  }
+                  __syncwarp();
+                }
+              }
+            }
+          }
+          tc_fence_before();
+      };
+      auto wait_q = [&]() {
+        if (!q_ready) {
+          const bool w = ok && mbar_wait_bounded(&bars->q_full[wg], qphase, abort_flag, status,
+                                                 kDevTimeoutAttn, TO);
+          qphase ^= 1;
+          q_ready = true;
+          ok = named_bar_and(1 + wg, 128, w);
+        }
+      };
       for (int pass = 0; pass < 3; ++pass) {
         // the third pass only runs for rows whose candidates overflowed (CTA-uniform decision)
         if (pass == 2 && !__syncthreads_or(overflow && scored && row < rows)) break;
         if (pass == 2) top.init(ksel);
+        if (ring) {
+          // Ring mode: piece k of the pass (past blocks k PR .. k PR + PR - 1) is ring load
+          // L0 + k, in slot (L0 + k) % RS. Thread 0 keeps RS loads in flight: load m + RS is
+          // issued once both warpgroups' products have finished reading load m (slot_free).
+          const int K_w = (n_self + C::PR - 1) / C::PR;  // pieces this warpgroup scores
+          const uint32_t L0 = ring_l;
+          if (tid == 0)
+            for (int k = 0; k < min(C::RS, K_pair); ++k) ring_load(L0 + k, k);
+          if (K_w > 0) wait_q();
+          auto issue_k = [&](int k) {
+            const uint32_t Lk = L0 + k;
+            const bool w = __all_sync(0xffffffffu,
+                                      ok && mbar_wait_bounded(&bars->slot_full[Lk % C::RS],
+                                                              (Lk / C::RS) & 1, abort_flag, status,
+                                                              kDevTimeoutAttn, TO));
+            if (w) issue_rows(static_cast<int>(Lk % C::RS) * C::PR,
+                              min(C::PR, n_self - k * C::PR), npiece & 1);
+          };
+          if (K_w > 0) {
+            if (ok && warp == wg * 4) issue_k(0);
+            ++npiece;
+          }
+          for (int k = 0; k < K_pair; ++k) {
+            const bool need = k < K_w;  // warpgroup-uniform
+            const uint32_t pc = npiece - 1;
+            if (need && k + 1 < K_w) {
+              if (ok && warp == wg * 4) issue_k(k + 1);
+              ++npiece;
+            }
+            bool w = ok;
+            if (need)
+              w = ok && mbar_wait_bounded(&bars->mma_done[wg][pc & 1], (pc >> 1) & 1, abort_flag,
+                                          status, kDevTimeoutAttn, TO);
+            // this warpgroup's products no longer read the slot (or never did). A warpgroup that
+            // does not score piece k still waits for its load first, so that its release counts
+            // toward this load and not an earlier one of the slot.
+            if (row == 0) {
+              const uint32_t Lk = L0 + k;
+              if (!need && ok)  // a timeout raises the abort flag; the release happens regardless
+                mbar_wait_bounded(&bars->slot_full[Lk % C::RS], (Lk / C::RS) & 1, abort_flag,
+                                  status, kDevTimeoutAttn, TO);
+              mbar_arrive(&bars->slot_free[Lk % C::RS]);
+            }
+            if (tid == 0 && k + C::RS < K_pair) ring_load(L0 + k + C::RS, k + C::RS);
+            if (need) {
+              if (__all_sync(0xffffffffu, w))
+                select_piece(pass, pc, k * C::PR, min(C::PR, n_self - k * C::PR));
+              // every thread of the warpgroup has read this buffer before piece k + 2 overwrites it
+              ok = named_bar_and(1 + wg, 128, w);
+            }
+          }
+          ring_l += K_pair;
+        } else {
         for (int ch = 0; ch < nchunks; ++ch) {
           const int c0 = ch * C::CAP;
           const int n = min(C::CAP, i_max - c0);
@@ -383,153 +621,26 @@ __global__ void __launch_bounds__(256, 1)
           }
           if (!scored || c0 >= i_t) continue;  // warpgroup-uniform
           const int n_t = min(n, i_t - c0);       // this tile's past blocks in the chunk
-          if (!q_ready) {
-            const bool w = ok && mbar_wait_bounded(&bars->q_full[wg], qphase, abort_flag, status,
-                                                   kDevTimeoutAttn, TO);
-            qphase ^= 1;
-            q_ready = true;
-            ok = named_bar_and(1 + wg, 128, w);
-          }
+          wait_q();
           // scores of this chunk, 128 past blocks per TMEM buffer; the products of piece p + 1 are
           // issued before piece p is selected (its buffer was freed by the barrier ending p - 1)
-          const uint32_t qa = smem_u32(sQ);
-          auto issue = [&](int p0) {  // one converged warp of the warpgroup issues
-            const int nmma = (min(C::PIECE, n_t - p0) + 15) & ~15;
-            const uint32_t idesc = idesc_bf16_f32(128, nmma, 0, 0);
-            const uint32_t buf = npiece & 1;
-            tc_fence_after();
-#pragma unroll
-            for (int sp = 0; sp < 2; ++sp) {
-#pragma unroll
-              for (int ks = 0; ks < D / 16; ++ks) {
-                const uint32_t aoff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                const uint32_t boff = static_cast<uint32_t>(sp * C::NCB * C::CAP * 128 +
-                                                            (ks >> 2) * C::CAP * 128 + p0 * 128 +
-                                                            (ks & 3) * 32);
-                mma_ss_elect(tmem + wg * 2 * C::PIECE + buf * C::PIECE,
-                             smem_desc_sw128(qa + aoff, 16, 1024),
-                             smem_desc_sw128(sBa + boff, 16, 1024), idesc,
-                             (sp > 0 || ks > 0) ? 1u : 0u);
-              }
-            }
-            mma_commit_elect(&bars->mma_done[wg][buf]);
-          };
-          if (ok && warp == wg * 4) issue(0);
+          if (ok && warp == wg * 4) issue_rows(0, min(C::PIECE, n_t), npiece & 1);
           ++npiece;
           for (int p0 = 0; p0 < n_t; p0 += C::PIECE) {
             const int np = min(C::PIECE, n_t - p0);
             const uint32_t pc = npiece - 1;  // this piece's number
             if (p0 + C::PIECE < n_t) {
-              if (ok && warp == wg * 4) issue(p0 + C::PIECE);
+              if (ok && warp == wg * 4)
+                issue_rows(p0 + C::PIECE, min(C::PIECE, n_t - p0 - C::PIECE), npiece & 1);
               ++npiece;
             }
             const bool w = ok && mbar_wait_bounded(&bars->mma_done[wg][pc & 1], (pc >> 1) & 1,
                                                    abort_flag, status, kDevTimeoutAttn, TO);
-            if (__all_sync(0xffffffffu, w)) {
-              tc_fence_after();
-              const uint32_t tb = t_s + (pc & 1) * C::PIECE;
-              // STEP columns per TMEM wait (64 with 32 groups, where both halves feed the same
-              // group maxima; 32 with 64 groups, for registers); columns past the tile's last past
-              // block read as -inf, so the per-score work below needs no bounds test
-              for (int cc = 0; cc < np; cc += STEP) {
-                uint32_t sa[32], sb[32];
-                const bool two = STEP == 64 && cc + 32 < np;  // warpgroup-uniform
-                tmem_ld32(tb + cc, sa);
-                if (two) tmem_ld32(tb + cc + 32, sb);
-                tmem_wait_ld();
-#pragma unroll
-                for (int x = 0; x < 32; ++x) {
-                  reg_fence(sa[x]);
-                  if (STEP == 64) reg_fence(sb[x]);
-                }
-                const int lim = np - cc;  // valid columns of the 64: c < lim
-                if (lim < STEP) {
-#pragma unroll
-                  for (int x = 0; x < 32; ++x) {
-                    if (x >= lim) sa[x] = __float_as_uint(-INFINITY);
-                    if (STEP == 64 && 32 + x >= lim) sb[x] = __float_as_uint(-INFINITY);
-                  }
-                }
-                const int jb = c0 + p0 + cc;  // block of sa[x] is jb + x, of sb[x] jb + 32 + x
-                if (pass == 0) {
-                  // group maxima, column j in group j mod M
-                  if (M == 32) {
-#pragma unroll
-                    for (int x = 0; x < 32; ++x)
-                      gmax[x] = fmax3(gmax[x], __uint_as_float(sa[x]), __uint_as_float(sb[x]));
-                  } else if ((jb & 32) == 0) {
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) gmax[x] = fmaxf(gmax[x], __uint_as_float(sa[x]));
-                  } else {
-#pragma unroll
-                    for (int x = 0; x < 32; ++x)
-                      gmax[(32 + x) % M] = fmaxf(gmax[(32 + x) % M], __uint_as_float(sa[x]));
-                  }
-                } else if (pass == 1) {
-                  // every score >= tau is a candidate, kept with its block (ascending). While at
-                  // least eight slots are free, eight columns at a time append without a capacity
-                  // test ((score, block) pairs to cand[slot][row]).
-                  auto append = [&](const uint32_t (&v)[32], int jb0) {
-#pragma unroll
-                    for (int x0 = 0; x0 < 32; x0 += 8) {
-                      if (cnt <= CB - 8) {
-                        uint32_t cp = cand_base + static_cast<uint32_t>(cnt) * 1024u;
-#pragma unroll
-                        for (int x = x0; x < x0 + 8; ++x)
-                          append_if_ge(cp, __uint_as_float(v[x]), tau, jb0 + x);
-                        cnt = static_cast<int>((cp - cand_base) >> 10);
-                      } else {
-#pragma unroll
-                        for (int x = x0; x < x0 + 8; ++x) {
-                          const float sv = __uint_as_float(v[x]);
-                          if (sv >= tau) {
-                            if (cnt < CB) {
-                              cand[cnt * 128 + row] = make_uint2(__float_as_uint(sv), jb0 + x);
-                            }
-                            ++cnt;
-                          }
-                        }
-                      }
-                    }
-                  };
-                  append(sa, jb);
-                  if (two) append(sb, jb + 32);
-                } else {
-                  // rows whose candidates overflowed keep a running top list instead
-#pragma unroll
-                  for (int hh = 0; hh < 2; ++hh) {
-                    if (hh == 1 && !two) break;
-                    const uint32_t(&sr)[32] = hh ? sb : sa;
-                    const int jh = jb + 32 * hh;
-                    const float thr0 = top.thr();
-                    uint32_t mask = 0;
-                    if (overflow) {
-#pragma unroll
-                      for (int x = 0; x < 32; ++x)
-                        if (__uint_as_float(sr[x]) > thr0) mask |= 1u << x;
-                    }
-                    if (__any_sync(0xffffffffu, mask != 0)) {
-                      if (overflow) {
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) cand[x * 128 + row].x = sr[x];
-                      }
-                      while (__any_sync(0xffffffffu, mask != 0)) {
-                        if (mask) {
-                          const int x = __ffs(mask) - 1;
-                          mask &= mask - 1;
-                          top.offer(__uint_as_float(cand[x * 128 + row].x), jh + x);
-                        }
-                      }
-                      __syncwarp();
-                    }
-                  }
-                }
-              }
-              tc_fence_before();
-            }
+            if (__all_sync(0xffffffffu, w)) select_piece(pass, pc, c0 + p0, np);
             // every thread of the warpgroup has read this buffer before piece p + 2 overwrites it
             ok = named_bar_and(1 + wg, 128, w);
           }
+        }
         }
         if (!scored) continue;
         if (pass == 0) {
@@ -624,6 +735,15 @@ __global__ void __launch_bounds__(256, 1)
     }
     ok = __syncthreads_and(ok);
     if (!ok) break;
+  }
+  if (tid == 0 && ring_issued > 0) {
+    // ring loads whose landing no wait may have seen: let them land before the CTA exits
+    volatile int no_abort = 0;
+    for (uint32_t x = 0; x < static_cast<uint32_t>(C::RS) && x < ring_issued; ++x) {
+      const uint32_t Lm = ring_issued - 1 - x;
+      mbar_wait_bounded(&bars->slot_full[Lm % C::RS], (Lm / C::RS) & 1, &no_abort, status,
+                        kDevDrainTimeout, kDrainTimeoutNs);
+    }
   }
   if (tid == 0 && chunk_pending) {
     // a chunk copy whose landing no wait saw: let it land before the CTA exits (bounded)

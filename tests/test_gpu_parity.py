@@ -129,10 +129,14 @@ def test_forward_small_all_rows(moba, case):
     ([0, 40000, 40000, 75000], 2, 1, 128, 128, 8),   # 313 + 274 blocks at d = 128: two chunks
     ([0, 70000], 2, 2, 64, 128, 20),                 # 547 blocks, k - 1 = 19: three chunks
     ([0, 30000, 64000], 4, 2, 64, 128, 5),           # 235 + 266 blocks, GQA
+    ([0, 80000], 2, 1, 64, 128, 16),                 # 625 blocks through a ring of four slots
+    ([0, 5000, 75000], 2, 2, 64, 128, 16),           # a resident unit, then ring units
+    ([0, 9000, 21000], 4, 2, 128, 128, 20),          # k - 1 = 19 at d = 128: 32-row ring slots
 ])
 def test_forward_many_blocks_sampled_rows(moba, cu, hq, hkv, d, B, topk):
     """Sequences of more than 257 blocks take the long-sequence gate, whose centroids the forward
-    pass splits into hi / lo once and copies in chunks; checked on sampled rows."""
+    pass splits into hi / lo once and keeps resident when they fit, else streams through a ring of
+    slots; checked on sampled rows."""
     w, q, k, v, cu_t = _inputs(cu, hq, hkv, d, B, topk, "clusters")
     tokens = wl.sample_tokens(w, 1024, seed=3)
     pu.run_and_check(moba, q, k, v, cu_t, cu, B, topk, 1.0 / math.sqrt(d), tokens=tokens)
