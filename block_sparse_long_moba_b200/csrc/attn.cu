@@ -35,10 +35,7 @@
 namespace moba {
 
 // Column pairs (of every 8) whose exp2 runs on the FMA pipe instead of MUFU.EX2, balancing the two.
-#ifndef MOBA_POLY_PAIRS_D64
-#define MOBA_POLY_PAIRS_D64 0
-#endif
-constexpr int kPolyPairs = MOBA_POLY_PAIRS_D64;
+constexpr int kPolyPairs = 0;
 #ifndef MOBA_POLY_PAIRS_PVT
 #define MOBA_POLY_PAIRS_PVT 1
 #endif
