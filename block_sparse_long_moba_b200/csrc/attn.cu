@@ -255,7 +255,8 @@ __global__ void __launch_bounds__(384, 1)
     attn_kernel_d64(const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v,
                     const __grid_constant__ CUtensorMap map_q,
-                    const __grid_constant__ CUtensorMap map_qd, const AttnArgs a) {
+                    const __grid_constant__ CUtensorMap map_qd,
+                    const __grid_constant__ CUtensorMap map_po, const AttnArgs a) {
   using C = D64Cfg;
   constexpr int D = C::D;
   extern __shared__ __align__(1024) uint8_t smem64[];
@@ -308,6 +309,7 @@ __global__ void __launch_bounds__(384, 1)
     prefetch_tensormap(&map_v);
     prefetch_tensormap(&map_q);
     prefetch_tensormap(&map_qd);
+    prefetch_tensormap(&map_po);
   }
   tc_fence_before();
   __syncthreads();
@@ -536,10 +538,12 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t t_o = tmem + lane_off + C::tm_o(half, ob);
       const int prev_prow = bars->ep_row[q];
       const float inv = bars->ep_inv[q];
-      // the warp's 32 output rows go through shared memory (16-byte chunk c of row r at chunk
-      // c ^ (r % 8), conflict-free both ways) and leave as whole 128-byte rows, four rows per warp
-      // instruction, instead of 32 scattered 16-byte pieces per instruction
+      // each thread's output row goes through shared memory (its 16-byte chunk c at chunk
+      // c ^ (r % 8) of the warp's staging row r: the 128-byte swizzle, conflict-free) and leaves
+      // as one 128-byte TMA store, so the warp does not wait for its stores; the staging row is
+      // reused one item later, once that store has read it
       uint8_t* ep = smem64 + C::OFF_EP + (warp - 4) * (32 * 128);
+      bulk_wait_group_read<0>();
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t orr[32];
@@ -556,17 +560,11 @@ __global__ void __launch_bounds__(384, 1)
               pack_bf16x2(__uint_as_float(orr[8 * x + 6]) * inv, __uint_as_float(orr[8 * x + 7]) * inv));
       }
       tc_fence_before();
-      __syncwarp();
-      const int c = lane & 7;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = 4 * i + (lane >> 3);
-        const int pr = __shfl_sync(0xffffffffu, prev_prow, r);
-        if (pr >= 0 && in_range(pr, a.rows_cap, a.status))
-          st_part(reinterpret_cast<uint4*>(a.part_o + static_cast<size_t>(pr) * D) + c,
-                  *reinterpret_cast<const uint4*>(ep + r * 128 + ((c ^ (r & 7)) * 16)));
+      if (prev_prow >= 0 && in_range(prev_prow, a.rows_cap, a.status)) {
+        fence_proxy_async_smem();  // the staging row is visible to the TMA unit
+        tma_store_2d(&map_po, ep + lane * 128, 0, prev_prow);
+        bulk_commit_group();
       }
-      __syncwarp();
       if (prev_prow >= 0 && in_range(prev_prow, a.rows_cap, a.status))
         a.part_lse[prev_prow] = bars->ep_lse[q];
       return true;
@@ -693,6 +691,7 @@ __global__ void __launch_bounds__(384, 1)
       ++ci;
     }
     if (ok && ci > 0) ok = epilogue();
+    bulk_wait_all();  // this thread's output stores are complete before the CTA exits
   }
 
   tc_fence_before();
@@ -1273,12 +1272,13 @@ static bool make_q_dense_map(CUtensorMap* map, const void* base, long long rows)
 }
 
 cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream) {
-  CUtensorMap mk, mv, mq, mqd;
+  CUtensorMap mk, mv, mq, mqd, mpo;
   if (!make_kv_map(&mk, L.k, L.T, L.G, L.d) || !make_kv_map(&mv, L.v, L.T, L.G, L.d))
     return cudaErrorInvalidValue;
   if (!make_q_rows_map(&mq, L.q, static_cast<long long>(L.T) * L.H, L.d))
     return cudaErrorInvalidValue;
-  if (L.d == 64 && (!L.qdense || !make_q_dense_map(&mqd, L.qdense, L.qdense_rows)))
+  if (L.d == 64 && (!L.qdense || !make_q_dense_map(&mqd, L.qdense, L.qdense_rows) ||
+                    !make_q_rows_map(&mpo, L.part_o, L.rows_cap, 64)))
     return cudaErrorInvalidValue;
   AttnArgs a;
   a.q = static_cast<const __nv_bfloat16*>(L.q);
@@ -1321,7 +1321,7 @@ cudaError_t launch_attention(const AttnLaunch& L, cudaStream_t stream) {
     const int smem = D64Cfg::SMEM_BYTES;
     cudaError_t e = cudaFuncSetAttribute(attn_kernel_d64, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_kernel_d64<<<grid, 384, smem, stream>>>(mk, mv, mq, mqd, a);
+    attn_kernel_d64<<<grid, 384, smem, stream>>>(mk, mv, mq, mqd, mpo, a);
   } else {
     const int smem = PvtCfg::SMEM_BYTES;
     cudaError_t e = cudaFuncSetAttribute(attn_kernel_pvt, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

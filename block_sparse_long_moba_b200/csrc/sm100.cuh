@@ -111,6 +111,26 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, u
       "r"(y3)
       : "memory");
 }
+// 2-D tiled store shared -> global of one box at element coordinates (x, y), tracked in this
+// thread's bulk async-group (x * element size a multiple of 16 bytes, y >= 0). No multicast.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until at most N of this thread's bulk async-groups still read their shared-memory source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Waits until all of this thread's bulk async-groups have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
 // Untiled bulk copy global -> shared of `bytes` (a multiple of 16; both addresses 16-byte
 // aligned), completion counted in bytes on `bar`. No multicast.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
