@@ -254,11 +254,15 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  // keys of this warp that lie in the chunk; the loop is unrolled with the loads predicated on it
+  // (not cut short), so several value rows are in flight at once
+  const int nk = max(0, min(64, u1 - (u0 + 64 * warp)));
+#pragma unroll 8
   for (int x = 0; x < 64; ++x) {
     const int src = x >> 1;
     const float p = __shfl_sync(0xffffffffu, (x & 1) ? p1 : p0, src);
-    const int u = u0 + 2 * (warp * 32 + src) + (x & 1);
-    if (u >= u1) break;  // uniform over the warp
+    if (x >= nk) continue;  // uniform over the warp
+    const int u = u0 + 64 * warp + x;  // key 2 (32 warp + src) + (x & 1) of the chunk
     const __nv_bfloat16* vr = v + static_cast<size_t>(u) * ld + g * D + lane * PER;
     if constexpr (PER == 4) {
       const uint2 w = __ldg(reinterpret_cast<const uint2*>(vr));
