@@ -211,8 +211,8 @@ __device__ __forceinline__ bool ring_consume(ItemRing* ring, uint32_t lt, Item& 
 //   * a routed item's query rows were densified in list order beforehand, so they arrive as one
 //     or two 128-row TMA tiles, QB items ahead;
 //   * O accumulators are double-buffered in TMEM per half (item parity), and the epilogue of an
-//     item runs after the next item's softmax, so it never delays the tensor pipe; it writes
-//     whole 128-byte rows through a per-warp staging area in shared memory;
+//     item runs after the next item's softmax, so it never delays the tensor pipe; each output
+//     row leaves a per-warp staging area in shared memory as one 128-byte TMA store;
 //   * an item of at most 128 rows (every diagonal item of a 128-key block, the tail item of a
 //     routed list) runs on half A only: half B issues no MMA and its warps skip the item.
 struct D64Cfg {

@@ -15,18 +15,21 @@
 //      largest group maximum tau is a lower bound of the ksel-th best score, since ksel distinct
 //      groups each hold a score >= tau;
 //   2. every score >= tau is a candidate (typically ksel + a few) and is appended, with its block,
-//      to the row's candidate buffer in shared memory (in ascending block order); a bitonic sort
-//      of the candidate scores gives the exact ksel-th best score tau* and how many selected
-//      scores tie with it, and a walk over the buffer writes the blocks with score > tau* and the
-//      lowest-numbered ones equal to tau* (ties go to the lower block), already ascending.
+//      to the row's candidate buffer in shared memory (one predicated 8-byte store per score, no
+//      branch; ascending block order); a bitonic sort of the candidate scores gives the exact
+//      ksel-th best score tau* and how many selected scores tie with it, the selection (the blocks
+//      with score > tau* and the lowest-numbered ones equal to tau*: ties go to the lower block)
+//      is marked in a bit mask, and the row is written ascending in 16-byte pieces.
 // Each pass costs a compare per score and no per-score list insertion. A row whose candidates
 // overflow the buffer (many exactly equal scores) runs a third pass with a running top list.
 //
 // A CTA holds two warpgroups (one query tile each) and works on one (query blocks, kv head) unit
 // at a time: the hi / lo centroids of the unit's past blocks are placed in shared memory once and
-// reused by all tiles of the unit when they fit, and streamed in chunks otherwise. Inside the
-// forward pass they come pre-split from global memory (one bulk copy per chunk and part, in the
-// swizzled row layout the MMA reads); the standalone gate converts the fp32 centroids itself.
+// reused by all tiles and passes of the unit when they fit. Inside the forward pass they come
+// pre-split from global memory (bulk copies in the swizzled row layout the MMA reads); when they
+// do not fit, they stream through a ring of slots, thread 0 issuing the load of a slot's next
+// piece as soon as both warpgroups' products have read it. The standalone gate converts the fp32
+// centroids itself, chunk by chunk.
 #include <algorithm>
 
 #include "common.cuh"
